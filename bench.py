@@ -1,0 +1,378 @@
+#!/usr/bin/env python
+"""Benchmark of one MoBA causal-prefill attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1m] [--impl ours|reference]
+
+One step = one full layer: block mean-pool, gate (scores, causal top-k, index
+build) and block-sparse attention with the merge, through the C ABI, on inputs
+already resident in HBM.  The metric is effective TFLOP/s on the algorithmic
+attention FLOPs (4 * head_dim per attended (query, key) pair), with ms per
+layer beside it.  With N > 1 (torchrun) every rank runs its own replica: the
+path has no exchange step, so there is no collective on the data path.
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import moba_synth as S  # noqa: E402
+
+METRIC = "MoBA prefill attn ms/layer & effective TFLOP/s (frac of bf16 TC peak) at 1M"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def algorithmic_pairs(cfg) -> int:
+    """Attended (query, key) pairs: sum over (b, h, t) of min(topk-1, c)*B + (t - cB + 1)."""
+    total = 0
+    for c in range((cfg.seqlen + cfg.block - 1) // cfg.block):
+        L = min(cfg.seqlen, (c + 1) * cfg.block) - c * cfg.block
+        total += min(cfg.topk - 1, c) * cfg.block * L + L * (L + 1) // 2
+    return total * cfg.batch * cfg.hq
+
+
+def attn_flops(cfg) -> float:
+    return 4.0 * cfg.head_dim * algorithmic_pairs(cfg)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        loaded = [x for x in sm if mx is None or x > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (the reference arm and the cpu_baseline leg)
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """The fp64 oracle on sampled query rows of the workload (one kv head)."""
+
+    def __init__(self, cfg, seed=0):
+        import numpy as np
+        import oracle as O
+        self.O, self.np, self.cfg = O, np, cfg
+        self.K = S.gen_head_rows(cfg, "k", 0, 0)
+        self.V = S.gen_head_rows(cfg, "v", 0, 0)
+        t0 = time.perf_counter()
+        self.kbar = O.mean_pool(self.K, cfg.block)
+        self.t_pool = time.perf_counter() - t0
+        self.rng = np.random.default_rng(seed)
+        self.Kd = None
+
+    def rows(self, n):
+        """Run n random rows; returns (seconds, attended pairs)."""
+        cfg, O, np = self.cfg, self.O, self.np
+        ts = self.rng.integers(0, cfg.seqlen, size=n)
+        hs = self.rng.integers(0, cfg.group, size=n)
+        qrows = [S.gen_rows(cfg, "q", 0, int(t), int(t) + 1, int(h))[0] for t, h in zip(ts, hs)]
+        pairs = 0
+        t0 = time.perf_counter()
+        for t, q in zip(ts, qrows):
+            out, lse, sel, gap = O.moba_row(q, self.K, self.V, self.kbar, int(t), cfg.block, cfg.topk,
+                                            cfg.softmax_scale)
+            pairs += len(O.key_positions(sel, int(t), cfg.block, cfg.seqlen))
+        return time.perf_counter() - t0, pairs
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 0) for p in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    smp = OracleSample(cfg)
+    secs, pairs, nrows = 0.0, 0, 0
+    while secs < budget_s and nrows < 20000:
+        s, p = smp.rows(16)
+        secs += s
+        pairs += p
+        nrows += 16
+    per_row = secs / nrows
+    total_rows = cfg.batch * cfg.seqlen * cfg.hq
+    full_s = per_row * total_rows + smp.t_pool * cfg.batch * cfg.hkv
+    return {
+        "value": attn_flops(cfg) / full_s / 1e12, "unit": "TFLOP/s",
+        "cores": blas_threads(), "kind": "oracle",
+        "sample": (f"{nrows} random query rows of the {cfg.name} layer (fp64 gather oracle, "
+                   f"{secs:.1f} s) plus the mean-pool of one kv head ({smp.t_pool:.1f} s), "
+                   f"extrapolated to the full layer"),
+        "extrapolated_full_layer_s": full_s, "sample_tflops": 4.0 * cfg.head_dim * pairs / secs / 1e12,
+    }
+
+
+def run_reference(args, cfg):
+    smp = OracleSample(cfg)
+    n = args.ref_rows
+    for _ in range(args.warmup):
+        smp.rows(n)
+    secs, pairs = 0.0, 0
+    for _ in range(args.steps):
+        s, p = smp.rows(n)
+        secs += s
+        pairs += p
+    value = 4.0 * cfg.head_dim * pairs / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(cfg, args),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{n} random query rows of the {cfg.name} layer per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(cfg, args):
+    return {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen, "hq": cfg.hq,
+            "hkv": cfg.hkv, "head_dim": cfg.head_dim, "block": cfg.block, "topk": cfg.topk,
+            "sparsity": 1.0 - algorithmic_pairs(cfg) / (cfg.batch * cfg.hq * cfg.seqlen *
+                                                       (cfg.seqlen + 1) / 2),
+            "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single",
+            "l2": "inputs larger than L2 (q alone 8.6 GB at 1M); no flush"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="1m", choices=sorted(S.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-rows", type=int, default=32)
+    args = ap.parse_args()
+    cfg = S.get_config(args.config)
+
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, cfg)
+        barrier(world)
+        return
+
+    import long_context_prefill_moba_b200 as M
+    M.load_library()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    q, k, v = S.gen_q(cfg, dev), S.gen_k(cfg, dev), S.gen_v(cfg, dev)
+    out = torch.empty_like(q)
+    layer = M.MobaLayer.from_config(cfg, dev)
+    sh = layer.shape
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        M.moba_block_meanpool(sh, k, layer.meank)
+        n = M.moba_last_launch_count()
+        if ev is not None:
+            ev[1].record(stream)
+        M.moba_gate_topk(sh, q, layer.meank, layer.sel, layer.offsets, layer.rows, layer.gate_ws)
+        n += M.moba_last_launch_count()
+        if ev is not None:
+            ev[2].record(stream)
+        M.moba_attn_fwd(sh, q, k, v, layer.sel, layer.offsets, layer.rows, out, None, layer.attn_ws)
+        n += M.moba_last_launch_count()
+        if ev is not None:
+            ev[3].record(stream)
+        return n
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(stream)
+    launches = 0
+    for i in range(args.steps):
+        launches += step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = start.elapsed_time(end) / args.steps
+    ms = max_over_ranks(ms, world)
+    pool_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    gate_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    flops = attn_flops(cfg)
+    value = world * flops / (ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    attn_tf = flops / (attn_ms * 1e-3) / 1e12
+    esz = 2 if cfg.dtype == "bf16" else 4
+    kbytes = cfg.batch * cfg.seqlen * cfg.hkv * cfg.head_dim * esz
+    qbytes = cfg.batch * cfg.seqlen * cfg.hq * cfg.head_dim * esz
+    pool_bytes = kbytes + layer.meank.numel() * 4
+    gate_bytes = qbytes + layer.sel.numel() * 4 * 2 + layer.rows.numel() * 4
+
+    # end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hq_, hk_, hv_ = (x.cpu().pin_memory() for x in (q, k, v))
+        ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            q.copy_(hq_, non_blocking=True)
+            k.copy_(hk_, non_blocking=True)
+            v.copy_(hv_, non_blocking=True)
+            launches_e2e = step()
+            ho.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
+        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 2 * kbytes + qbytes, "d2h_bytes_per_step": qbytes}
+        del hq_, hk_, hv_, ho
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, args.cpu_budget)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": config_of(cfg, args),
+            "ms_per_layer": ms,
+            "kernels_ms": {"meanpool": pool_ms, "gate": gate_ms, "attn": attn_ms},
+            "roofline": {"bound": "tensor", "kernel": "moba_attn_fwd (attention + merge)",
+                         "achieved": attn_tf, "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
+                         "peak_kind": f"{peak_kind} bf16 sustained", "traffic": None},
+            "hbm_kernels": {
+                "meanpool": {"achieved": pool_bytes / (pool_ms * 1e-3) / 1e9, "unit": "GB/s",
+                             "peak": peaks["hbm_gbs"]},
+                "gate": {"achieved": gate_bytes / (gate_ms * 1e-3) / 1e9, "unit": "GB/s",
+                         "peak": peaks["hbm_gbs"]}},
+            "whole_step_frac_of_peak": (flops / (ms * 1e-3) / 1e12) / peaks["bf16_tflops"],
+            "gpu_launches": launches,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

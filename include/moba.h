@@ -1,0 +1,191 @@
+/*
+ * moba.h — C ABI of the MoBA (Mixture of Block Attention) causal-prefill
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * Method: "MoBA: Mixture of Block Attention for Long-Context LLMs"
+ * (arXiv 2502.13189).  Section names below are those of the paper-graph
+ * summary page of that paper ([summary]); [note] is the research-hub concept
+ * note "MoBA (Mixture of Block Attention)", "Key math / How it works"; [review]
+ * is the paperhub.cn OpenReview discussion page of the paper (reviews and
+ * author rebuttals).
+ *
+ * The forward pass is three calls on one CUDA stream:
+ *   moba_block_meanpool  pooled key of every size-B block      ([summary] §3
+ *                        "Affinity Scoring"; Algorithm 1 Step 1)
+ *   moba_gate_topk       causal top-k block selection per query head plus the
+ *                        query-per-block index                  ([summary] §3
+ *                        "Top-k Gating", "Causality Enforcement"; Algorithm 1
+ *                        Steps 1-2)
+ *   moba_attn_fwd        softmax attention over the union of the selected
+ *                        blocks, causal inside the current block, with the
+ *                        online-softmax merge                   ([summary] §3
+ *                        "The Core MoBA Attention Equation"; Algorithm 1
+ *                        Steps 3-4)
+ *
+ * Conventions shared by every call
+ *   - Tensors are dense and contiguous: q and out [batch, seqlen, hq, head_dim],
+ *     k and v [batch, seqlen, hkv, head_dim].  q, k, v and out share the dtype
+ *     (bf16 or fp32).  All pointers are DEVICE pointers on the current device,
+ *     16-byte aligned.
+ *   - The caller owns all memory.  The library never allocates or frees device
+ *     memory, keeps no state between calls and never synchronises: every call
+ *     only enqueues work on `stream` and returns.
+ *   - Arguments are validated before anything is enqueued.  A bad argument
+ *     returns MOBA_ERR_INVALID_ARG / MOBA_ERR_UNSUPPORTED / MOBA_ERR_WORKSPACE
+ *     and launches nothing.  A launch failure returns MOBA_ERR_CUDA (the CUDA
+ *     error code is available from moba_last_cuda_error()).  Errors that
+ *     happen later on the device surface through the stream as usual.
+ *   - topk counts the current block: each query attends to its own block
+ *     (causally) plus the top (topk-1) earlier blocks by unscaled <q, mean K>.
+ *     Equal scores go to the lower block index.  Future blocks are never
+ *     selected.  With fewer than topk-1 earlier blocks, all are selected.
+ *   - GQA: query head h uses kv head h / (hq / hkv); every query head selects
+ *     its own blocks ([review] rebuttal W1 on the OpenReview discussion page).
+ *   - seqlen need not be a multiple of block: the last block is shorter.
+ *   - scale <= 0 selects 1/sqrt(head_dim).  lse is the natural-log
+ *     log-sum-exp of the scaled logits.
+ *   - Sizes: seqlen*hq*batch < 2^31 and head_dim in {64, 128};
+ *     1 <= topk <= MOBA_MAX_TOPK.
+ */
+#ifndef MOBA_H_
+#define MOBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOBA_API __attribute__((visibility("default")))
+#else
+#define MOBA_API
+#endif
+
+typedef struct CUstream_st* moba_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+#define MOBA_MAX_TOPK 16
+
+typedef enum {
+  MOBA_OK = 0,
+  MOBA_ERR_INVALID_ARG = 1,  /* null pointer, misaligned pointer, bad shape   */
+  MOBA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. head_dim 96) */
+  MOBA_ERR_WORKSPACE = 3,    /* workspace smaller than the *_workspace_size  */
+  MOBA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed         */
+  MOBA_ERR_INTERNAL = 5,
+  MOBA_ERR_TIMEOUT = 6       /* reserved: a bounded device-side wait expired */
+} moba_status_t;
+
+typedef enum { MOBA_BF16 = 0, MOBA_F32 = 1 } moba_dtype_t;
+
+typedef struct {
+  int32_t batch;       /* independent sequences                                   */
+  int32_t seqlen;      /* N: tokens per sequence                                  */
+  int32_t hq;          /* query heads                                             */
+  int32_t hkv;         /* key/value heads; hq % hkv == 0                          */
+  int32_t head_dim;    /* d: 64 or 128                                            */
+  int32_t block;       /* B: tokens per KV block                                  */
+  int32_t topk;        /* blocks attended per query, counting the current block  */
+  int32_t dtype;       /* moba_dtype_t of q, k, v and out                         */
+  float scale;         /* softmax scale; <= 0 selects 1/sqrt(head_dim)           */
+  int32_t query_chunk; /* tokens per attention pass; 0 = automatic (see below)   */
+} moba_shape_t;
+
+/* ---- sizes (host only, no CUDA calls) --------------------------------- */
+
+/* MOBA_OK if the shape is supported, else the status moba_* calls return. */
+MOBA_API moba_status_t moba_check_shape(const moba_shape_t* shape);
+
+/* n = ceil(seqlen / block). */
+MOBA_API int64_t moba_num_blocks(const moba_shape_t* shape);
+
+/* Tokens per attention pass C.  The query range is processed in passes of C
+ * tokens (for every batch entry at once) so that the per-block partial
+ * results of one pass fit a bounded workspace.  query_chunk > 0 (a multiple
+ * of 128) is used as given; 0 picks the largest power of two >= 128 whose
+ * partials fit 8 GiB, capped at seqlen rounded up to 128. */
+MOBA_API int64_t moba_query_chunk(const moba_shape_t* shape);
+
+/* Number of passes: ceil(seqlen / C). */
+MOBA_API int64_t moba_num_chunks(const moba_shape_t* shape);
+
+/* Elements of meank: batch * n * hkv * head_dim (fp32). */
+MOBA_API int64_t moba_meank_elems(const moba_shape_t* shape);
+
+/* Elements of sel: batch * seqlen * hq * topk (int32). */
+MOBA_API int64_t moba_sel_elems(const moba_shape_t* shape);
+
+/* Elements of offsets: num_chunks * batch * hkv * n + 1 (int32). */
+MOBA_API int64_t moba_offsets_elems(const moba_shape_t* shape);
+
+/* Exact number of rows entries: batch * hq * sum_t min(topk-1, t / block). */
+MOBA_API int64_t moba_rows_elems(const moba_shape_t* shape);
+
+/* Device scratch bytes needed by moba_gate_topk / moba_attn_fwd. */
+MOBA_API size_t moba_gate_workspace_size(const moba_shape_t* shape);
+MOBA_API size_t moba_attn_workspace_size(const moba_shape_t* shape);
+
+/* ---- the three steps --------------------------------------------------- */
+
+/* Block mean-pool ([summary] §3 "Affinity Scoring": the block representation
+ * mean_pool(K[I_i]), computed once per layer; Algorithm 1 Step 1).
+ *   k      [batch, seqlen, hkv, head_dim]  dtype     (read)
+ *   meank  [batch, n, hkv, head_dim]       fp32      (written)
+ * meank[b,j,g,:] is the mean of k[b, t, g, :] over the rows t of block j
+ * (a shorter last block is averaged over its own rows). */
+MOBA_API moba_status_t moba_block_meanpool(const moba_shape_t* shape, const void* k, float* meank,
+                                           moba_stream_t stream);
+
+/* Gate ([summary] §3 "Top-k Gating" g_i = 1[s_i in Topk], "Causality
+ * Enforcement" mechanism 1, the current block as a shared expert; Algorithm 1
+ * Step 1 S = Q meanK^T with the causal mask, and Step 2 grouping queries by
+ * block).
+ *   q        [batch, seqlen, hq, head_dim]  dtype   (read)
+ *   meank    output of moba_block_meanpool          (read)
+ *   sel      [batch, seqlen, hq, topk] int32        (written) selected blocks
+ *            of each query head, ascending; the current block is the last
+ *            valid entry; unused entries are -1.
+ *   offsets  [moba_offsets_elems] int32             (written) exclusive
+ *            prefix over groups (chunk, b, kv head g, block j) in that order:
+ *            rows[offsets[i] .. offsets[i+1]) are the query rows of pass
+ *            `chunk` that selected earlier block j and read kv head g.
+ *   rows     [moba_rows_elems] int32                (written) query row ids
+ *            r = (b * seqlen + t) * hq + h (the row of q viewed as
+ *            [batch*seqlen*hq, head_dim]); within a group the order is
+ *            unspecified.
+ *   ws       >= moba_gate_workspace_size bytes of device scratch. */
+MOBA_API moba_status_t moba_gate_topk(const moba_shape_t* shape, const void* q, const float* meank,
+                                      int32_t* sel, int32_t* offsets, int32_t* rows, void* ws,
+                                      size_t ws_bytes, moba_stream_t stream);
+
+/* Block-sparse attention ([summary] §3 "The Core MoBA Attention Equation"
+ * MoBA(q,K,V) = Softmax(q K[I]^T) V[I]; "Causality Enforcement" mechanism 2,
+ * causal inside the current block; Algorithm 1 Step 3 (history without mask,
+ * grouped by block so each block's K/V serves all its queries) and Step 4
+ * (online-softmax merge of the partial results)).
+ *   q, k, v            as above                              (read)
+ *   sel, offsets, rows outputs of moba_gate_topk             (read)
+ *   out   [batch, seqlen, hq, head_dim] dtype                (written)
+ *   lse   [batch, hq, seqlen] fp32, natural log, or NULL     (written)
+ *   ws    >= moba_attn_workspace_size bytes of device scratch. */
+MOBA_API moba_status_t moba_attn_fwd(const moba_shape_t* shape, const void* q, const void* k,
+                                     const void* v, const int32_t* sel, const int32_t* offsets,
+                                     const int32_t* rows, void* out, float* lse, void* ws,
+                                     size_t ws_bytes, moba_stream_t stream);
+
+/* ---- diagnostics ------------------------------------------------------- */
+
+/* Static description of a status code. */
+MOBA_API const char* moba_status_string(moba_status_t status);
+
+/* The cudaError_t behind the last MOBA_ERR_CUDA returned on this thread. */
+MOBA_API int moba_last_cuda_error(void);
+
+/* Number of kernel launches the last moba_* call on this thread enqueued. */
+MOBA_API int moba_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOBA_H_ */

@@ -1,0 +1,233 @@
+"""MoBA (Mixture of Block Attention) causal prefill on NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/moba.h`` (``libmoba.so``, built
+in-tree by ``long_context_prefill_moba_b200.build``).  Every step of the
+computation runs in the library's CUDA kernels; this module only marshals
+torch tensors (device memory and the current CUDA stream) into the C calls.
+There is no CPU fallback: if the library is missing, importing the functions
+raises.
+
+Functions with the names of the C entry points:
+
+    moba_block_meanpool(shape, k, meank)
+    moba_gate_topk(shape, q, meank, sel, offsets, rows, ws)
+    moba_attn_fwd(shape, q, k, v, sel, offsets, rows, out, lse, ws)
+
+plus ``MobaLayer`` (owns the intermediate buffers of one shape and runs the
+three steps) and ``moba_forward`` (allocating convenience call).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "MobaShape", "MobaError", "lib", "load_library", "make_shape", "moba_check_shape",
+    "moba_num_blocks", "moba_query_chunk", "moba_num_chunks", "moba_meank_elems",
+    "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems", "moba_gate_workspace_size",
+    "moba_attn_workspace_size", "moba_block_meanpool", "moba_gate_topk", "moba_attn_fwd",
+    "moba_status_string", "moba_last_launch_count", "MobaLayer", "moba_forward",
+    "MOBA_BF16", "MOBA_F32", "EXPORTED_SYMBOLS",
+]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoba.so")
+
+MOBA_BF16, MOBA_F32 = 0, 1
+MOBA_OK = 0
+
+EXPORTED_SYMBOLS = [
+    "moba_check_shape", "moba_num_blocks", "moba_query_chunk", "moba_num_chunks",
+    "moba_meank_elems", "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems",
+    "moba_gate_workspace_size", "moba_attn_workspace_size", "moba_block_meanpool",
+    "moba_gate_topk", "moba_attn_fwd", "moba_status_string", "moba_last_cuda_error",
+    "moba_last_launch_count",
+]
+
+
+class MobaShape(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("seqlen", ctypes.c_int32), ("hq", ctypes.c_int32),
+        ("hkv", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32),
+        ("topk", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float),
+        ("query_chunk", ctypes.c_int32),
+    ]
+
+    def __repr__(self):
+        return "MobaShape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class MobaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = lib().moba_status_string(status).decode()
+        if status == 4:
+            msg += f" (cudaError {lib().moba_last_cuda_error()})"
+        super().__init__(f"{where}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libmoba.so and declare its signatures (raises if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m long_context_prefill_moba_b200.build` (no CPU fallback exists)")
+    L = ctypes.CDLL(path)
+    P = ctypes.POINTER(MobaShape)
+    vp, i64, sz, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+    for name in ("moba_num_blocks", "moba_query_chunk", "moba_num_chunks", "moba_meank_elems",
+                 "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems"):
+        getattr(L, name).argtypes = [P]
+        getattr(L, name).restype = i64
+    for name in ("moba_gate_workspace_size", "moba_attn_workspace_size"):
+        getattr(L, name).argtypes = [P]
+        getattr(L, name).restype = sz
+    L.moba_check_shape.argtypes = [P]
+    L.moba_check_shape.restype = st
+    L.moba_block_meanpool.argtypes = [P, vp, vp, vp]
+    L.moba_block_meanpool.restype = st
+    L.moba_gate_topk.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moba_gate_topk.restype = st
+    L.moba_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moba_attn_fwd.restype = st
+    L.moba_status_string.argtypes = [st]
+    L.moba_status_string.restype = ctypes.c_char_p
+    L.moba_last_cuda_error.argtypes = []
+    L.moba_last_cuda_error.restype = st
+    L.moba_last_launch_count.argtypes = []
+    L.moba_last_launch_count.restype = st
+    _lib = L
+    return L
+
+
+def lib():
+    return load_library()
+
+
+def make_shape(batch, seqlen, hq, hkv, head_dim, block, topk, dtype="bf16", scale=None,
+               query_chunk=0) -> MobaShape:
+    dt = {"bf16": MOBA_BF16, torch.bfloat16: MOBA_BF16, "f32": MOBA_F32, torch.float32: MOBA_F32}[dtype]
+    return MobaShape(batch, seqlen, hq, hkv, head_dim, block, topk, dt,
+                     0.0 if scale is None else float(scale), query_chunk)
+
+
+def _s(shape):
+    return ctypes.byref(shape)
+
+
+def moba_check_shape(shape) -> int: return lib().moba_check_shape(_s(shape))
+def moba_num_blocks(shape) -> int: return lib().moba_num_blocks(_s(shape))
+def moba_query_chunk(shape) -> int: return lib().moba_query_chunk(_s(shape))
+def moba_num_chunks(shape) -> int: return lib().moba_num_chunks(_s(shape))
+def moba_meank_elems(shape) -> int: return lib().moba_meank_elems(_s(shape))
+def moba_sel_elems(shape) -> int: return lib().moba_sel_elems(_s(shape))
+def moba_offsets_elems(shape) -> int: return lib().moba_offsets_elems(_s(shape))
+def moba_rows_elems(shape) -> int: return lib().moba_rows_elems(_s(shape))
+def moba_gate_workspace_size(shape) -> int: return lib().moba_gate_workspace_size(_s(shape))
+def moba_attn_workspace_size(shape) -> int: return lib().moba_attn_workspace_size(_s(shape))
+def moba_status_string(status: int) -> str: return lib().moba_status_string(status).decode()
+def moba_last_launch_count() -> int: return lib().moba_last_launch_count()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the MoBA library must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != MOBA_OK:
+        raise MobaError(status, where)
+
+
+def moba_block_meanpool(shape, k, meank, stream=None):
+    _check(lib().moba_block_meanpool(_s(shape), _ptr(k), _ptr(meank), _stream(stream)),
+           "moba_block_meanpool")
+
+
+def moba_gate_topk(shape, q, meank, sel, offsets, rows, ws, stream=None):
+    _check(lib().moba_gate_topk(_s(shape), _ptr(q), _ptr(meank), _ptr(sel), _ptr(offsets), _ptr(rows),
+                                _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moba_gate_topk")
+
+
+def moba_attn_fwd(shape, q, k, v, sel, offsets, rows, out, lse, ws, stream=None):
+    _check(lib().moba_attn_fwd(_s(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(offsets),
+                               _ptr(rows), _ptr(out), _ptr(lse), _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)),
+           "moba_attn_fwd")
+
+
+class MobaLayer:
+    """Buffers of one MoBA layer shape on one device, and the three steps.
+
+    ``forward(q, k, v, out, lse=None)`` enqueues mean-pool, gate and attention
+    on the current stream.  Intermediate results stay readable afterwards:
+    ``meank``, ``sel``, ``offsets``, ``rows``."""
+
+    def __init__(self, batch, seqlen, hq, hkv, head_dim, block, topk, dtype="bf16", scale=None,
+                 query_chunk=0, device="cuda"):
+        self.shape = make_shape(batch, seqlen, hq, hkv, head_dim, block, topk, dtype, scale,
+                                query_chunk)
+        _check(moba_check_shape(self.shape), "MobaLayer")
+        dev = torch.device(device)
+        self.device = dev
+        i32 = torch.int32
+        self.meank = torch.empty(moba_meank_elems(self.shape), dtype=torch.float32, device=dev)
+        self.sel = torch.empty(moba_sel_elems(self.shape), dtype=i32, device=dev)
+        self.offsets = torch.empty(moba_offsets_elems(self.shape), dtype=i32, device=dev)
+        self.rows = torch.empty(max(1, moba_rows_elems(self.shape)), dtype=i32, device=dev)
+        self.gate_ws = torch.empty(moba_gate_workspace_size(self.shape), dtype=torch.uint8, device=dev)
+        self.attn_ws = torch.empty(moba_attn_workspace_size(self.shape), dtype=torch.uint8, device=dev)
+        self.launches = 0
+
+    @classmethod
+    def from_config(cls, cfg, device="cuda", query_chunk=0):
+        return cls(cfg.batch, cfg.seqlen, cfg.hq, cfg.hkv, cfg.head_dim, cfg.block, cfg.topk,
+                   cfg.dtype, cfg.scale, query_chunk, device)
+
+    def forward(self, q, k, v, out, lse=None, stream=None):
+        s = self.shape
+        moba_block_meanpool(s, k, self.meank, stream)
+        n = moba_last_launch_count()
+        moba_gate_topk(s, q, self.meank, self.sel, self.offsets, self.rows, self.gate_ws, stream)
+        n += moba_last_launch_count()
+        moba_attn_fwd(s, q, k, v, self.sel, self.offsets, self.rows, out, lse, self.attn_ws, stream)
+        n += moba_last_launch_count()
+        self.launches = n
+        return out
+
+    def sel_view(self):
+        s = self.shape
+        return self.sel.view(s.batch, s.seqlen, s.hq, s.topk)
+
+    def meank_view(self):
+        s = self.shape
+        return self.meank.view(s.batch, moba_num_blocks(s), s.hkv, s.head_dim)
+
+
+def moba_forward(q, k, v, block, topk, scale=None, return_lse=False, query_chunk=0):
+    """out (and lse) of one MoBA layer; q [b,N,Hq,d], k/v [b,N,Hkv,d] CUDA tensors."""
+    b, N, hq, d = q.shape
+    layer = MobaLayer(b, N, hq, k.shape[2], d, block, topk, q.dtype, scale, query_chunk, q.device)
+    out = torch.empty_like(q)
+    lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device) if return_lse else None
+    layer.forward(q, k, v, out, lse)
+    return (out, lse) if return_lse else out

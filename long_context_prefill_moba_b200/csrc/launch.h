@@ -1,0 +1,38 @@
+// Host-side launchers of the MoBA kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moba {
+
+// Every launcher enqueues on `stream`, adds the kernels it launched to
+// *launches and returns the first CUDA error seen (cudaSuccess otherwise).
+
+// rows entries contributed by tokens [t0, t1) of one (b, h): sum min(KH, t / B)
+int64_t hist_rows_range(int64_t t0, int64_t t1, int64_t B, int64_t KH);
+
+cudaError_t launch_meanpool(const Dims& dm, int dtype, const void* k, float* meank,
+                            cudaStream_t stream, int* launches);
+
+struct GateWs {
+  int32_t* counts;   // [ngroups] rows per (chunk, b, g, j)
+  int32_t* cursors;  // [ngroups] scatter cursors
+};
+cudaError_t launch_gate(const Dims& dm, int dtype, const void* q, const float* meank, int32_t* sel,
+                        int32_t* offsets, int32_t* rows, GateWs ws, cudaStream_t stream,
+                        int* launches);
+
+struct AttnWs {
+  float* part_o;        // [b * C * hq * (topk-1), d]  normalised partial outputs
+  float* part_lse;      // [b * C * hq * (topk-1)]     their log2-sum-exp2
+  int32_t* tile_start;  // [b * hkv * n + 1]           tile prefix of one pass
+};
+cudaError_t launch_attn(const Dims& dm, int dtype, const void* q, const void* k, const void* v,
+                        const int32_t* sel, const int32_t* offsets, const int32_t* rows, void* out,
+                        float* lse, AttnWs ws, cudaStream_t stream, int* launches);
+
+}  // namespace moba

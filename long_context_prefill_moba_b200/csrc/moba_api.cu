@@ -1,0 +1,218 @@
+// C ABI of the MoBA causal-prefill forward: argument validation, sizes and the
+// three entry points declared in include/moba.h.
+#include <math.h>
+
+#include "launch.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+thread_local int g_last_launches = 0;
+
+constexpr int64_t kI32Max = 2147483647;
+constexpr int64_t kPartialBudget = 8ll << 30;   // bytes of partials per pass (automatic chunk)
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int64_t nblocks(const moba_shape_t* s) { return ((int64_t)s->seqlen + s->block - 1) / s->block; }
+
+int64_t chunk_of(const moba_shape_t* s) {
+  const int64_t cap = round_up(s->seqlen, 128);
+  if (s->query_chunk > 0) return s->query_chunk < cap ? s->query_chunk : cap;
+  const int64_t KH = s->topk - 1;
+  if (KH == 0) return cap;
+  const int64_t per_token = (int64_t)s->batch * s->hq * KH * (s->head_dim + 1) * 4;
+  int64_t c = 128;
+  while (c * 2 <= cap && c * 2 * per_token <= kPartialBudget) c *= 2;
+  return c < cap ? c : cap;
+}
+
+int64_t nchunks_of(const moba_shape_t* s) {
+  const int64_t c = chunk_of(s);
+  return (s->seqlen + c - 1) / c;
+}
+
+int64_t ngroups_total(const moba_shape_t* s) {
+  return nchunks_of(s) * s->batch * s->hkv * nblocks(s);
+}
+
+int64_t rows_total(const moba_shape_t* s) {
+  return moba::hist_rows_range(0, s->seqlen, s->block, s->topk - 1) * s->batch * s->hq;
+}
+
+moba::Dims make_dims(const moba_shape_t* s) {
+  moba::Dims d;
+  d.batch = s->batch;
+  d.N = s->seqlen;
+  d.hq = s->hq;
+  d.hkv = s->hkv;
+  d.d = s->head_dim;
+  d.B = s->block;
+  d.topk = s->topk;
+  d.n = (int)nblocks(s);
+  d.G = s->hq / s->hkv;
+  d.chunk = (int)chunk_of(s);
+  d.nchunks = (int)nchunks_of(s);
+  const float scale = s->scale > 0.f ? s->scale : 1.0f / sqrtf((float)s->head_dim);
+  d.scale_log2 = scale * moba::kLog2e;
+  return d;
+}
+
+size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct AttnLayout {
+  size_t part_o, part_lse, tile_start, total;
+};
+AttnLayout attn_layout(const moba_shape_t* s) {
+  const size_t KH = s->topk - 1;
+  const size_t entries = (size_t)s->batch * chunk_of(s) * s->hq * KH;
+  AttnLayout L;
+  L.part_o = 0;
+  L.part_lse = L.part_o + align_up(entries * s->head_dim * sizeof(float));
+  L.tile_start = L.part_lse + align_up(entries * sizeof(float));
+  L.total = L.tile_start + align_up(((size_t)s->batch * s->hkv * nblocks(s) + 1) * sizeof(int32_t));
+  return L;
+}
+
+moba_status_t finish(cudaError_t e, int launches) {
+  g_last_launches = launches;
+  if (e != cudaSuccess) {
+    g_last_cuda_error = (int)e;
+    return MOBA_ERR_CUDA;
+  }
+  return MOBA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+MOBA_API moba_status_t moba_check_shape(const moba_shape_t* s) {
+  if (s == nullptr) return MOBA_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->seqlen < 1 || s->hq < 1 || s->hkv < 1 || s->block < 1 || s->topk < 1 ||
+      s->head_dim < 1)
+    return MOBA_ERR_INVALID_ARG;
+  if (s->hq % s->hkv != 0) return MOBA_ERR_INVALID_ARG;
+  if (s->dtype != MOBA_BF16 && s->dtype != MOBA_F32) return MOBA_ERR_INVALID_ARG;
+  if (isnan(s->scale) || isinf(s->scale)) return MOBA_ERR_INVALID_ARG;
+  if (s->query_chunk < 0 || (s->query_chunk > 0 && s->query_chunk % 128 != 0))
+    return MOBA_ERR_INVALID_ARG;
+  if (s->head_dim != 64 && s->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
+  if (s->topk > MOBA_MAX_TOPK) return MOBA_ERR_UNSUPPORTED;
+  if ((int64_t)s->batch * s->seqlen * s->hq > kI32Max) return MOBA_ERR_UNSUPPORTED;
+  if (rows_total(s) > kI32Max) return MOBA_ERR_UNSUPPORTED;
+  if (ngroups_total(s) + 1 > kI32Max) return MOBA_ERR_UNSUPPORTED;
+  if ((int64_t)s->batch * chunk_of(s) * s->hq * (s->topk - 1) > kI32Max) return MOBA_ERR_UNSUPPORTED;
+  return MOBA_OK;
+}
+
+MOBA_API int64_t moba_num_blocks(const moba_shape_t* s) {
+  return moba_check_shape(s) == MOBA_OK ? nblocks(s) : -1;
+}
+MOBA_API int64_t moba_query_chunk(const moba_shape_t* s) {
+  return moba_check_shape(s) == MOBA_OK ? chunk_of(s) : -1;
+}
+MOBA_API int64_t moba_num_chunks(const moba_shape_t* s) {
+  return moba_check_shape(s) == MOBA_OK ? nchunks_of(s) : -1;
+}
+MOBA_API int64_t moba_meank_elems(const moba_shape_t* s) {
+  return moba_check_shape(s) == MOBA_OK ? (int64_t)s->batch * nblocks(s) * s->hkv * s->head_dim : -1;
+}
+MOBA_API int64_t moba_sel_elems(const moba_shape_t* s) {
+  return moba_check_shape(s) == MOBA_OK ? (int64_t)s->batch * s->seqlen * s->hq * s->topk : -1;
+}
+MOBA_API int64_t moba_offsets_elems(const moba_shape_t* s) {
+  return moba_check_shape(s) == MOBA_OK ? ngroups_total(s) + 1 : -1;
+}
+MOBA_API int64_t moba_rows_elems(const moba_shape_t* s) {
+  return moba_check_shape(s) == MOBA_OK ? rows_total(s) : -1;
+}
+MOBA_API size_t moba_gate_workspace_size(const moba_shape_t* s) {
+  if (moba_check_shape(s) != MOBA_OK) return 0;
+  return align_up(2 * (size_t)ngroups_total(s) * sizeof(int32_t));
+}
+MOBA_API size_t moba_attn_workspace_size(const moba_shape_t* s) {
+  if (moba_check_shape(s) != MOBA_OK) return 0;
+  return attn_layout(s).total;
+}
+
+MOBA_API moba_status_t moba_block_meanpool(const moba_shape_t* s, const void* k, float* meank,
+                                           moba_stream_t stream) {
+  g_last_launches = 0;
+  moba_status_t st = moba_check_shape(s);
+  if (st != MOBA_OK) return st;
+  if (k == nullptr || meank == nullptr || !aligned16(k) || !aligned16(meank))
+    return MOBA_ERR_INVALID_ARG;
+  int launches = 0;
+  cudaError_t e = moba::launch_meanpool(make_dims(s), s->dtype, k, meank, (cudaStream_t)stream,
+                                        &launches);
+  return finish(e, launches);
+}
+
+MOBA_API moba_status_t moba_gate_topk(const moba_shape_t* s, const void* q, const float* meank,
+                                      int32_t* sel, int32_t* offsets, int32_t* rows, void* ws,
+                                      size_t ws_bytes, moba_stream_t stream) {
+  g_last_launches = 0;
+  moba_status_t st = moba_check_shape(s);
+  if (st != MOBA_OK) return st;
+  if (q == nullptr || meank == nullptr || sel == nullptr || offsets == nullptr || ws == nullptr)
+    return MOBA_ERR_INVALID_ARG;
+  if (rows == nullptr && rows_total(s) > 0) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(meank) || !aligned4(sel) || !aligned4(offsets) ||
+      (rows != nullptr && !aligned4(rows)) || !aligned16(ws))
+    return MOBA_ERR_INVALID_ARG;
+  if (ws_bytes < moba_gate_workspace_size(s)) return MOBA_ERR_WORKSPACE;
+  const int64_t L = ngroups_total(s);
+  moba::GateWs g{static_cast<int32_t*>(ws), static_cast<int32_t*>(ws) + L};
+  int launches = 0;
+  cudaError_t e = moba::launch_gate(make_dims(s), s->dtype, q, meank, sel, offsets, rows, g,
+                                    (cudaStream_t)stream, &launches);
+  return finish(e, launches);
+}
+
+MOBA_API moba_status_t moba_attn_fwd(const moba_shape_t* s, const void* q, const void* k,
+                                     const void* v, const int32_t* sel, const int32_t* offsets,
+                                     const int32_t* rows, void* out, float* lse, void* ws,
+                                     size_t ws_bytes, moba_stream_t stream) {
+  g_last_launches = 0;
+  moba_status_t st = moba_check_shape(s);
+  if (st != MOBA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || sel == nullptr || offsets == nullptr ||
+      out == nullptr || ws == nullptr)
+    return MOBA_ERR_INVALID_ARG;
+  if (rows == nullptr && rows_total(s) > 0) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(sel) ||
+      !aligned4(offsets) || (rows != nullptr && !aligned4(rows)) || !aligned16(ws) ||
+      (lse != nullptr && !aligned4(lse)))
+    return MOBA_ERR_INVALID_ARG;
+  if (ws_bytes < moba_attn_workspace_size(s)) return MOBA_ERR_WORKSPACE;
+  AttnLayout L = attn_layout(s);
+  char* base = static_cast<char*>(ws);
+  moba::AttnWs a{reinterpret_cast<float*>(base + L.part_o), reinterpret_cast<float*>(base + L.part_lse),
+                 reinterpret_cast<int32_t*>(base + L.tile_start)};
+  int launches = 0;
+  cudaError_t e = moba::launch_attn(make_dims(s), s->dtype, q, k, v, sel, offsets, rows, out, lse, a,
+                                    (cudaStream_t)stream, &launches);
+  return finish(e, launches);
+}
+
+MOBA_API const char* moba_status_string(moba_status_t st) {
+  switch (st) {
+    case MOBA_OK: return "MOBA_OK";
+    case MOBA_ERR_INVALID_ARG: return "MOBA_ERR_INVALID_ARG: invalid argument";
+    case MOBA_ERR_UNSUPPORTED: return "MOBA_ERR_UNSUPPORTED: shape or dtype not supported";
+    case MOBA_ERR_WORKSPACE: return "MOBA_ERR_WORKSPACE: workspace too small";
+    case MOBA_ERR_CUDA: return "MOBA_ERR_CUDA: CUDA launch or runtime error";
+    case MOBA_ERR_INTERNAL: return "MOBA_ERR_INTERNAL: internal error";
+    case MOBA_ERR_TIMEOUT: return "MOBA_ERR_TIMEOUT: device wait timed out";
+  }
+  return "unknown moba_status_t";
+}
+
+MOBA_API int moba_last_cuda_error(void) { return g_last_cuda_error; }
+MOBA_API int moba_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

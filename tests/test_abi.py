@@ -1,0 +1,122 @@
+"""The C-ABI library loads, exports every symbol include/moba.h declares, and
+validates its arguments on the host (no compute call needs a GPU here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_prefill_moba_b200 as M
+from long_context_prefill_moba_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moba.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return M.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MOBA_API\s+[\w\s\*]*?\b(moba_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_symbols() == sorted(M.EXPORTED_SYMBOLS)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_no_other_symbols_are_exported(L):
+    out = os.popen(f"nm -D --defined-only {M.LIB_PATH}").read()
+    ours = sorted({ln.split()[-1] for ln in out.splitlines() if " T " in ln and "moba" in ln})
+    assert ours == declared_symbols()
+
+
+def shape(**kw):
+    base = dict(batch=1, seqlen=1 << 20, hq=32, hkv=8, head_dim=128, block=4096, topk=12,
+                dtype="bf16", scale=None, query_chunk=0)
+    base.update(kw)
+    return M.make_shape(**base)
+
+
+def test_sizes_of_the_1m_layer(L):
+    s = shape()
+    assert M.moba_check_shape(s) == 0
+    assert M.moba_num_blocks(s) == 256
+    C = M.moba_query_chunk(s)
+    assert C % 128 == 0 and C * 32 * 11 * 129 * 4 <= 8 << 30
+    assert M.moba_num_chunks(s) == (1 << 20) // C
+    assert M.moba_sel_elems(s) == (1 << 20) * 32 * 12
+    assert M.moba_meank_elems(s) == 256 * 8 * 128
+    assert M.moba_offsets_elems(s) == M.moba_num_chunks(s) * 8 * 256 + 1
+    # rows: sum_t min(11, t // 4096) per head
+    exact = sum(min(11, c) * 4096 for c in range(256)) * 32
+    assert M.moba_rows_elems(s) == exact
+    assert M.moba_attn_workspace_size(s) >= C * 32 * 11 * 129 * 4
+    assert M.moba_gate_workspace_size(s) >= 2 * 4 * M.moba_num_chunks(s) * 8 * 256
+
+
+def test_rows_count_ragged_and_small(L):
+    s = shape(batch=2, seqlen=1000, hq=4, hkv=2, block=96, topk=3)
+    exact = sum(min(2, t // 96) for t in range(1000)) * 2 * 4
+    assert M.moba_rows_elems(s) == exact
+    s1 = shape(batch=1, seqlen=100, hq=2, hkv=1, block=128, topk=4)
+    assert M.moba_rows_elems(s1) == 0 and M.moba_num_blocks(s1) == 1
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), 1), (dict(seqlen=0), 1), (dict(hq=6, hkv=4), 1), (dict(block=0), 1),
+    (dict(topk=0), 1), (dict(dtype="f32", head_dim=96), 2), (dict(topk=17), 2),
+    (dict(query_chunk=100), 1), (dict(scale=float("nan")), 1),
+    (dict(batch=64, seqlen=1 << 20, hq=64), 2),
+])
+def test_invalid_shapes_rejected(L, kw, status):
+    s = shape(**kw)
+    assert M.moba_check_shape(s) == status
+    assert M.moba_num_blocks(s) == -1
+    assert M.moba_attn_workspace_size(s) == 0
+
+
+def test_entry_points_validate_before_launching(L):
+    s = shape(seqlen=4096, block=256)
+    fake = ctypes.c_void_p(1 << 20)          # never dereferenced: validation fails first
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    P = ctypes.byref(s)
+    # null / misaligned pointers
+    assert L.moba_block_meanpool(P, None, fake, None) == 1
+    assert L.moba_block_meanpool(P, odd, fake, None) == 1
+    # workspace too small
+    assert L.moba_gate_topk(P, fake, fake, fake, fake, fake, fake, 16, None) == 3
+    assert L.moba_attn_fwd(P, fake, fake, fake, fake, fake, fake, fake, None, fake, 16, None) == 3
+    # bad shape
+    bad = shape(hq=5, hkv=2)
+    assert L.moba_attn_fwd(ctypes.byref(bad), fake, fake, fake, fake, fake, fake, fake, None, fake,
+                           1 << 40, None) == 1
+    assert L.moba_gate_topk(None, fake, fake, fake, fake, fake, fake, 1 << 40, None) == 1
+    assert L.moba_last_launch_count() == 0
+
+
+def test_status_strings(L):
+    for st in range(7):
+        assert M.moba_status_string(st).startswith("MOBA_")
+    assert "unknown" in M.moba_status_string(99)
+
+
+def test_library_missing_fails_loudly(tmp_path):
+    import importlib
+    mod = importlib.reload(M)
+    saved = mod._lib
+    try:
+        mod._lib = None
+        with pytest.raises(RuntimeError, match="no CPU fallback"):
+            mod.load_library(str(tmp_path / "libmoba.so"))
+    finally:
+        mod._lib = saved
