@@ -185,6 +185,35 @@ MOBA_API int moba_last_cuda_error(void);
 /* Number of kernel launches the last moba_* call on this thread enqueued. */
 MOBA_API int moba_last_launch_count(void);
 
+/* ---- gate without caller-provided scratch ----------------------------- */
+
+/* Groups (offsets entries minus one) the allocation-free gate can index. */
+#define MOBA_GATE_NOALLOC_MAX_GROUPS (1 << 19)
+
+/* moba_gate_topk for callers that cannot hand the library any device scratch:
+ * for example a plain C host program that has no device allocator of its own,
+ * or a serving runtime that reserves all device memory when it starts and
+ * forbids allocations afterwards.  The paper has no counterpart: this is a
+ * packaging variant of the gate, not a step of the method.
+ *
+ * Same arguments, results and layouts as moba_gate_topk, minus ws/ws_bytes.
+ * The scratch (two int32 counters per group) lives in a fixed array inside
+ * the library: 2 * MOBA_GATE_NOALLOC_MAX_GROUPS int32 (4 MiB), held on every
+ * GPU that loads the library until the process exits.  Shapes with more than
+ * MOBA_GATE_NOALLOC_MAX_GROUPS groups (moba_offsets_elems - 1) are rejected
+ * with MOBA_ERR_UNSUPPORTED before anything is enqueued.
+ *   - Nothing is allocated: no cudaMalloc/cudaFree and no allocating library
+ *     routine.  The counters are cleared on `stream` at the start of every call.
+ *   - The first call on each device looks up that device's address of the
+ *     array (with the device current); make that first call before any stream
+ *     capture on the device.
+ *   - All calls on a device share the one array: calls that overlap on the GPU
+ *     (different streams without ordering between them) race and give wrong
+ *     results.  Order them on one stream or with events. */
+MOBA_API moba_status_t moba_gate_topk_noalloc(const moba_shape_t* shape, const void* q,
+                                              const float* meank, int32_t* sel, int32_t* offsets,
+                                              int32_t* rows, moba_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -30,7 +30,7 @@ __all__ = [
     "moba_num_blocks", "moba_query_chunk", "moba_num_chunks", "moba_meank_elems",
     "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems", "moba_gate_workspace_size",
     "moba_attn_workspace_size", "moba_block_meanpool", "moba_gate_topk", "moba_attn_fwd",
-    "moba_status_string", "moba_last_launch_count", "MobaLayer", "moba_forward",
+    "moba_status_string", "moba_last_launch_count", "moba_gate_topk_noalloc", "MobaLayer", "moba_forward",
     "MOBA_BF16", "MOBA_F32", "EXPORTED_SYMBOLS",
 ]
 
@@ -45,7 +45,7 @@ EXPORTED_SYMBOLS = [
     "moba_meank_elems", "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems",
     "moba_gate_workspace_size", "moba_attn_workspace_size", "moba_block_meanpool",
     "moba_gate_topk", "moba_attn_fwd", "moba_status_string", "moba_last_cuda_error",
-    "moba_last_launch_count",
+    "moba_last_launch_count", "moba_gate_topk_noalloc",
 ]
 
 
@@ -99,6 +99,8 @@ def load_library(path: str = LIB_PATH):
     L.moba_gate_topk.restype = st
     L.moba_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moba_attn_fwd.restype = st
+    L.moba_gate_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
+    L.moba_gate_topk_noalloc.restype = st
     L.moba_status_string.argtypes = [st]
     L.moba_status_string.restype = ctypes.c_char_p
     L.moba_last_cuda_error.argtypes = []
@@ -166,6 +168,15 @@ def moba_gate_topk(shape, q, meank, sel, offsets, rows, ws, stream=None):
     _check(lib().moba_gate_topk(_s(shape), _ptr(q), _ptr(meank), _ptr(sel), _ptr(offsets), _ptr(rows),
                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "moba_gate_topk")
+
+
+def moba_gate_topk_noalloc(shape, q, meank, sel, offsets, rows, stream=None):
+    """moba_gate_topk without caller scratch: the counters live in a fixed
+    device array inside the library (for callers that cannot give the library
+    device scratch memory).  Calls on one device must not overlap on the GPU."""
+    _check(lib().moba_gate_topk_noalloc(_s(shape), _ptr(q), _ptr(meank), _ptr(sel), _ptr(offsets),
+                                        _ptr(rows), _stream(stream)),
+           "moba_gate_topk_noalloc")
 
 
 def moba_attn_fwd(shape, q, k, v, sel, offsets, rows, out, lse, ws, stream=None):

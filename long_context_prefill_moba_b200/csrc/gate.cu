@@ -286,3 +286,52 @@ cudaError_t launch_gate(const Dims& dm, int dtype, const void* q, const float* m
 }
 
 }  // namespace moba
+
+// ---------------------------------------------------------------------------
+// Allocation-free gate: the scratch counters live in a fixed device array of
+// this file instead of caller-provided memory (see moba_gate_topk_noalloc).
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+static __device__ __align__(256) int32_t g_gate_scratch[2 * MOBA_GATE_NOALLOC_MAX_GROUPS];
+
+std::mutex g_scratch_mu;
+int32_t* g_scratch_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_gate_scratch on the current device (looked up once per
+// device; the host-side symbol itself is not a device address).
+cudaError_t scratch_for_current_device(int32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_gate_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+namespace moba {
+
+cudaError_t launch_gate_noalloc(const Dims& dm, int dtype, const void* q, const float* meank,
+                                int32_t* sel, int32_t* offsets, int32_t* rows,
+                                cudaStream_t stream, int* launches) {
+  int32_t* scratch = nullptr;
+  cudaError_t e = scratch_for_current_device(&scratch);
+  if (e != cudaSuccess) return e;
+  const int64_t L = (int64_t)dm.nchunks * dm.batch * dm.hkv * dm.n;
+  GateWs ws{scratch, scratch + L};   // counts, then cursors; launch_gate clears both
+  return launch_gate(dm, dtype, q, meank, sel, offsets, rows, ws, stream, launches);
+}
+
+}  // namespace moba

@@ -26,6 +26,12 @@ cudaError_t launch_gate(const Dims& dm, int dtype, const void* q, const float* m
                         int32_t* offsets, int32_t* rows, GateWs ws, cudaStream_t stream,
                         int* launches);
 
+// moba_gate_topk with the counters in the library's fixed device array
+// (requires nchunks * batch * hkv * n <= MOBA_GATE_NOALLOC_MAX_GROUPS)
+cudaError_t launch_gate_noalloc(const Dims& dm, int dtype, const void* q, const float* meank,
+                                int32_t* sel, int32_t* offsets, int32_t* rows,
+                                cudaStream_t stream, int* launches);
+
 struct AttnWs {
   float* part_o;        // [b * C * hq * (topk-1), d]  normalised partial outputs
   float* part_lse;      // [b * C * hq * (topk-1)]     their log2-sum-exp2

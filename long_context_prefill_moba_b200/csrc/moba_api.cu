@@ -199,6 +199,25 @@ MOBA_API moba_status_t moba_attn_fwd(const moba_shape_t* s, const void* q, const
   return finish(e, launches);
 }
 
+MOBA_API moba_status_t moba_gate_topk_noalloc(const moba_shape_t* s, const void* q,
+                                              const float* meank, int32_t* sel, int32_t* offsets,
+                                              int32_t* rows, moba_stream_t stream) {
+  g_last_launches = 0;
+  moba_status_t st = moba_check_shape(s);
+  if (st != MOBA_OK) return st;
+  if (ngroups_total(s) > MOBA_GATE_NOALLOC_MAX_GROUPS) return MOBA_ERR_UNSUPPORTED;
+  if (q == nullptr || meank == nullptr || sel == nullptr || offsets == nullptr)
+    return MOBA_ERR_INVALID_ARG;
+  if (rows == nullptr && rows_total(s) > 0) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(meank) || !aligned4(sel) || !aligned4(offsets) ||
+      (rows != nullptr && !aligned4(rows)))
+    return MOBA_ERR_INVALID_ARG;
+  int launches = 0;
+  cudaError_t e = moba::launch_gate_noalloc(make_dims(s), s->dtype, q, meank, sel, offsets, rows,
+                                            (cudaStream_t)stream, &launches);
+  return finish(e, launches);
+}
+
 MOBA_API const char* moba_status_string(moba_status_t st) {
   switch (st) {
     case MOBA_OK: return "MOBA_OK";
