@@ -13,6 +13,10 @@ cudaError_t launch_attn_mma_hist(const Dims& dm, const void* q, const void* k, c
 cudaError_t launch_attn_mma_cur(const Dims& dm, const void* q, const void* k, const void* v,
                                 const AttnWs& ws, void* out, float* lse, int ch,
                                 cudaStream_t stream);
+cudaError_t launch_attn_tc_hist(const Dims& dm, const void* q, const void* k, const void* v,
+                                const int32_t* sel, const int32_t* offsets, const int32_t* rows,
+                                const AttnWs& ws, int ch, int64_t grid, cudaStream_t stream);
+int attn_tc_rows_per_tile();
 cudaError_t launch_attn_f32_hist(const Dims& dm, const void* q, const void* k, const void* v,
                                  const int32_t* sel, const int32_t* offsets, const int32_t* rows,
                                  const AttnWs& ws, int ch, int64_t nrows, cudaStream_t stream);
@@ -37,21 +41,26 @@ cudaError_t launch_attn(const Dims& dm, int dtype, const void* q, const void* k,
                         float* lse, AttnWs ws, cudaStream_t stream, int* launches) {
   const int KH = dm.topk - 1;
   const int ngroups = dm.batch * dm.hkv * dm.n;
-  cudaError_t e = cudaSuccess;
+  cudaError_t e = cudaMemsetAsync(ws.status, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return e;
+  // bf16 with head_dim 128: tensor-core (tcgen05) kernel for the historical blocks
+  const bool tc = dtype == MOBA_BF16 && dm.d == 128;
+  const int tm = tc ? attn_tc_rows_per_tile() : 64;
   for (int ch = 0; ch < dm.nchunks; ++ch) {
     const int t0 = ch * dm.chunk;
     const int t1 = dm.N < t0 + dm.chunk ? dm.N : t0 + dm.chunk;
     const int64_t nrows = hist_rows_range(t0, t1, dm.B, KH) * dm.batch * dm.hq;
     if (nrows > 0) {
       if (dtype == MOBA_BF16) {
-        attn_plan_kernel<<<1, 1024, 0, stream>>>(offsets + (size_t)ch * ngroups, ngroups, 64,
+        attn_plan_kernel<<<1, 1024, 0, stream>>>(offsets + (size_t)ch * ngroups, ngroups, tm,
                                                  ws.tile_start);
         ++*launches;
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const int cmax = (t1 - 1) / dm.B;
         const int64_t active = (int64_t)dm.batch * dm.hkv * (cmax < dm.n ? cmax : dm.n);
-        const int64_t grid = nrows / 64 + active + 1;
-        e = launch_attn_mma_hist(dm, q, k, v, sel, offsets, rows, ws, ch, grid, stream);
+        const int64_t grid = nrows / tm + active + 1;
+        e = tc ? launch_attn_tc_hist(dm, q, k, v, sel, offsets, rows, ws, ch, grid, stream)
+               : launch_attn_mma_hist(dm, q, k, v, sel, offsets, rows, ws, ch, grid, stream);
       } else {
         e = launch_attn_f32_hist(dm, q, k, v, sel, offsets, rows, ws, ch, nrows, stream);
       }

@@ -1,0 +1,400 @@
+// K3a on 5th-generation tensor cores (tcgen05 + TMEM + TMA): attention of the
+// grouped queries over one earlier ("historical") block, no mask.
+//
+// "MoBA: Mixture of Block Attention for Long-Context LLMs", paper-graph summary
+// §3 "The Core MoBA Attention Equation" and Implementation, Algorithm 1 Step 3:
+// the queries that routed to a block are gathered so that the block's keys and
+// values are loaded once for all of them; the per-row partial results are
+// merged later with the current-block part (Step 4).
+//
+// One CTA = one work tile of up to 256 query rows of one (b, kv head g, block j)
+// group, as two 128-row tiles Q0 / Q1 (TMEM lanes = rows).  Roles:
+//   warps 0-3  softmax for Q0        warps 4-7  softmax for Q1
+//   warp 8     TMA producer of K/V tiles (and TMEM allocation)
+//   warp 9     single-thread tcgen05.mma issuer      warps 10-11 idle
+// The softmax warpgroups raise their register budget to 216 with setmaxnreg
+// and the third warpgroup drops to 64 (384 x 168 at launch = 256 x 216 + 128 x 64
+// + 1024 spare).
+// Per 128-key tile i: S_w = Q_w K_i^T (SS MMA, fp32 in TMEM), the softmax warps
+// read S_w, keep a lazily rescaled running max, write P_w = exp2(S - m) as bf16
+// back over S_w, and O_w += P_w V_i runs as a TS MMA (A operand from TMEM).
+// TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) columns.
+// SMEM: Q0 Q1 (32 KB each), K and V double buffered (32 KB per tile): 192 KB.
+// All tiles use the 128-byte swizzled K-major layout (V is read MN-major).
+//
+// The MMA issue order per tile i is PV0_i, S0_{i+1}, PV1_i, S1_{i+1}; tcgen05
+// operations of one thread execute in order and a commit covers every earlier
+// operation, so when S_w(i+1) is signalled complete, PV_w(i) is complete too and
+// the softmax warps may rescale O_w in place before releasing P_w(i+1).
+//
+// Every wait is bounded (2 s); on expiry the CTA drains what it issued, frees
+// TMEM and reports MOBA_ERR_TIMEOUT through the status word.
+#include <cudaTypedefs.h>
+
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace moba {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kQT = 128;                 // rows per Q tile
+constexpr int kBK = 128;                 // keys per K/V tile
+constexpr int kRowsPerCta = 2 * kQT;
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;     // registers per thread at launch (ptxas, 384 threads, 1 CTA/SM)
+constexpr int kSoftmaxRegs = 216;
+constexpr int kServiceRegs = 64;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kServiceRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+constexpr uint32_t kTile = kBK * kD * 2; // 32 KB, two 16 KB column halves
+constexpr uint32_t kHalf = 16384;
+constexpr uint32_t kOffQ = 0;            // Q0 at 0, Q1 at kTile
+constexpr uint32_t kOffK = 2 * kTile;    // stages at +0, +kTile
+constexpr uint32_t kOffV = 4 * kTile;
+constexpr uint32_t kSmemBytes = 6 * kTile + 1024;
+constexpr float kRescaleThreshold = 8.f; // log2 units: rescale O only when the max grows by > 2^8
+
+struct Ctl {
+  uint64_t q_full[2], k_full[2], v_full[2], k_free[2], v_free[2], s_full[2], p_full[2], o_full[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+MOBA_DEV uint32_t bar(const uint64_t* b) { return smem_u32(b); }
+
+__global__ void __launch_bounds__(kThreads, 1) attn_hist_tc_kernel(
+    const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap tmK,
+    const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ sel,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ rows,
+    const int32_t* __restrict__ tile_start, float* __restrict__ part_o,
+    float* __restrict__ part_lse, int* __restrict__ status, Dims dm, int ch) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ Ctl ctl;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+
+  const int ngroups = dm.batch * dm.hkv * dm.n;
+  const int tile = blockIdx.x;
+  if (tile >= tile_start[ngroups]) return;
+  int lo = 0, hi = ngroups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  const int grp = lo;
+  const int j = grp % dm.n;
+  const int g = (grp / dm.n) % dm.hkv;
+  const int b = grp / (dm.n * dm.hkv);
+  const size_t goff = (size_t)ch * ngroups + grp;
+  const int r0 = offsets[goff] + (tile - tile_start[grp]) * kRowsPerCta;
+  const int cnt = min(kRowsPerCta, offsets[goff + 1] - r0);
+  const int nq = cnt > kQT ? 2 : 1;
+  const int nkt = (dm.B + kBK - 1) / kBK;
+  const int KH = dm.topk - 1;
+  const int t0 = ch * dm.chunk;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(bar(&ctl.q_full[w]), kQT);
+      mbar_init(bar(&ctl.p_full[w]), kQT);
+      mbar_init(bar(&ctl.k_full[w]), 1);
+      mbar_init(bar(&ctl.v_full[w]), 1);
+      mbar_init(bar(&ctl.k_free[w]), 1);
+      mbar_init(bar(&ctl.v_free[w]), 1);
+      mbar_init(bar(&ctl.s_full[w]), 1);
+      mbar_init(bar(&ctl.o_full[w]), 1);
+    }
+    mbar_init(bar(&ctl.drain), 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(&ctl.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = ctl.tmem_base;
+  volatile int* abort_flag = &ctl.abort;
+  if (warp < 8)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
+  else
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kServiceRegs));
+
+  if (warp < 8) {
+    // ------------------------------------------------------------ softmax
+    const int w = warp >> 2;
+    if (w < nq) {
+      const int rho = tid & 127;
+      const int row_i = w * kQT + rho;
+      const bool valid = row_i < cnt;
+      const int r = valid ? rows[r0 + row_i] : 0;
+      const uint32_t qs = base + kOffQ + w * kTile;
+      const __nv_bfloat16* src = q + (size_t)r * kD;
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        cp_async16(qs + (c >> 3) * kHalf + sw128_off(rho, c & 7), src + c * 8, valid);
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(bar(&ctl.q_full[w]));
+      size_t pidx = 0;
+      if (valid) {
+        const int h = r % dm.hq;
+        const int t = (r / dm.hq) % dm.N;
+        const int slot = slot_of(sel + (size_t)r * dm.topk, dm.topk, j);
+        pidx = (size_t)((b * dm.chunk + (t - t0)) * dm.hq + h) * KH + slot;
+      }
+      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t tS = tb + (w ? 128u : 0u) + lane_off;
+      const uint32_t tO = tb + (w ? 384u : 256u) + lane_off;
+      const float sl2 = dm.scale_log2;
+      float m_used = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int i = 0; i < nkt && ok; ++i) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.s_full[w]), i & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld32(tS + 0, sr);
+        tmem_ld32(tS + 32, sr + 32);
+        tmem_ld32(tS + 64, sr + 64);
+        tmem_ld32(tS + 96, sr + 96);
+        tmem_wait_ld();
+        const int kvalid = dm.B - i * kBK;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          float x = __uint_as_float(sr[c]);
+          if (c >= kvalid) x = -INFINITY;
+          sr[c] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+        const float mxs = mx * sl2;
+        const bool need = mxs > m_used + kRescaleThreshold;
+        if (i > 0 && __any_sync(0xffffffffu, need)) {
+          const float f = need ? exp2f(m_used - mxs) : 1.f;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(tO + cc * 32, o);
+          }
+          tmem_wait_st();
+        }
+        if (need) {
+          l *= exp2f(m_used - mxs);
+          m_used = mxs;
+        }
+        float rs = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = exp2f(fmaf(__uint_as_float(sr[2 * c]), sl2, -m_used));
+          const float p1 = exp2f(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m_used));
+          rs += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l += rs;
+        tmem_st32(tS + 0, pk);
+        tmem_st32(tS + 32, pk + 32);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(&ctl.p_full[w]));
+      }
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.o_full[w]), 0, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        float* dst = part_o + pidx * kD;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_wait_ld();
+          if (valid) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dst + cc * 32 + e) =
+                  make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                              __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          }
+        }
+        if (valid) part_lse[pidx] = m_used + log2f(l);
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const int y0 = b * dm.N + j * dm.B;
+      const int x0 = g * kD;
+      int issued_k = 0, issued_v = 0;
+      for (int i = 0; i < nkt; ++i) {
+        const int s = i & 1;
+        const uint32_t ks = base + kOffK + s * kTile, vs = base + kOffV + s * kTile;
+        if (i >= 2 && !mbar_wait(bar(&ctl.k_free[s]), ((i >> 1) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(&ctl.k_full[s]), kTile);
+        tma_load_2d(ks, &tmK, x0, y0 + i * kBK, bar(&ctl.k_full[s]));
+        tma_load_2d(ks + kHalf, &tmK, x0 + 64, y0 + i * kBK, bar(&ctl.k_full[s]));
+        issued_k = i + 1;
+        if (i >= 2 && !mbar_wait(bar(&ctl.v_free[s]), ((i >> 1) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(&ctl.v_full[s]), kTile);
+        tma_load_2d(vs, &tmV, x0, y0 + i * kBK, bar(&ctl.v_full[s]));
+        tma_load_2d(vs + kHalf, &tmV, x0 + 64, y0 + i * kBK, bar(&ctl.v_full[s]));
+        issued_v = i + 1;
+      }
+      if (*abort_flag) {
+        // let the copies this thread issued land before the CTA exits
+        int never = 0;
+        for (int i = (issued_k > 2 ? issued_k - 2 : 0); i < issued_k; ++i)
+          mbar_wait(bar(&ctl.k_full[i & 1]), (i >> 1) & 1, &never);
+        for (int i = (issued_v > 2 ? issued_v - 2 : 0); i < issued_v; ++i)
+          mbar_wait(bar(&ctl.v_full[i & 1]), (i >> 1) & 1, &never);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16(128, kBK, false);
+      const uint32_t idO = idesc_bf16(128, kD, true);
+      auto issue_s = [&](int w, int s) {
+        const uint32_t qa = base + kOffQ + w * kTile, ka = base + kOffK + s * kTile;
+        const uint32_t d = tb + (w ? 128u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          mma_ss(d, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int w, int s, bool acc) {
+        const uint32_t va = base + kOffV + s * kTile;
+        const uint32_t d = tb + (w ? 384u : 256u), a = tb + (w ? 128u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(d, a + kk * 8, sdesc_sw128(va + kk * 2048, kHalf, 1024), idO, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar(&ctl.q_full[0]), 0, abort_flag);
+      if (ok && nq == 2) ok = mbar_wait(bar(&ctl.q_full[1]), 0, abort_flag);
+      if (ok) ok = mbar_wait(bar(&ctl.k_full[0]), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        mma_commit(bar(&ctl.s_full[0]));
+        if (nq == 2) {
+          issue_s(1, 0);
+          mma_commit(bar(&ctl.s_full[1]));
+        }
+        mma_commit(bar(&ctl.k_free[0]));
+      }
+      for (int i = 0; i < nkt && ok; ++i) {
+        const int s = i & 1, s1 = (i + 1) & 1;
+        const bool more = i + 1 < nkt;
+        ok = mbar_wait(bar(&ctl.v_full[s]), (i >> 1) & 1, abort_flag) &&
+             mbar_wait(bar(&ctl.p_full[0]), i & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, s, i > 0);
+        if (more) {
+          if (!(ok = mbar_wait(bar(&ctl.k_full[s1]), ((i + 1) >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_s(0, s1);
+          mma_commit(bar(&ctl.s_full[0]));
+        }
+        if (nq == 2) {
+          if (!(ok = mbar_wait(bar(&ctl.p_full[1]), i & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(1, s, i > 0);
+          if (more) {
+            issue_s(1, s1);
+            mma_commit(bar(&ctl.s_full[1]));
+          }
+        }
+        mma_commit(bar(&ctl.v_free[s]));
+        if (more) mma_commit(bar(&ctl.k_free[s1]));
+      }
+      if (ok) {
+        mma_commit(bar(&ctl.o_full[0]));
+        if (nq == 2) mma_commit(bar(&ctl.o_full[1]));
+      } else {
+        // drain every MMA this thread issued before TMEM is released
+        int never = 0;
+        mma_commit(bar(&ctl.drain));
+        mbar_wait(bar(&ctl.drain), 0, &never);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 8) tmem_dealloc(tb, 512);
+  if (tid == 0 && ctl.abort) atomicExch(status, (int)MOBA_ERR_TIMEOUT);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a [batch*N, hkv*d] bf16 tensor, 128 rows x 64 columns per box,
+// 128-byte swizzle; rows past the end read as zero.
+bool make_kv_map(CUtensorMap* map, const void* base, const Dims& dm) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)dm.hkv * kD, (cuuint64_t)dm.batch * dm.N};
+  cuuint64_t strides[1] = {(cuuint64_t)dm.hkv * kD * 2};
+  cuuint32_t box[2] = {64, kBK};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+constexpr int kTcRowsPerTile = kRowsPerCta;
+
+cudaError_t launch_attn_tc_hist(const Dims& dm, const void* q, const void* k, const void* v,
+                                const int32_t* sel, const int32_t* offsets, const int32_t* rows,
+                                const AttnWs& ws, int ch, int64_t grid, cudaStream_t stream) {
+  CUtensorMap mk, mv;
+  if (!make_kv_map(&mk, k, dm) || !make_kv_map(&mv, v, dm)) return cudaErrorInvalidValue;
+  // the setmaxnreg split is only safe if the kernel really launches with kLaunchRegs
+  static int launch_regs = -1;
+  if (launch_regs < 0) {
+    cudaFuncAttributes fa;
+    cudaError_t ea = cudaFuncGetAttributes(&fa, attn_hist_tc_kernel);
+    if (ea != cudaSuccess) return ea;
+    launch_regs = fa.numRegs;
+  }
+  if (launch_regs < kLaunchRegs) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(attn_hist_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemBytes);
+  if (e != cudaSuccess) return e;
+  attn_hist_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
+      (const __nv_bfloat16*)q, mk, mv, sel, offsets, rows, ws.tile_start, ws.part_o, ws.part_lse,
+      ws.status, dm, ch);
+  return cudaGetLastError();
+}
+
+int attn_tc_rows_per_tile() { return kTcRowsPerTile; }
+
+}  // namespace moba

@@ -33,6 +33,7 @@ cudaError_t launch_gate_noalloc(const Dims& dm, int dtype, const void* q, const 
                                 cudaStream_t stream, int* launches);
 
 struct AttnWs {
+  int* status;          // device status word: 0, or MOBA_ERR_TIMEOUT after a bounded wait expired
   float* part_o;        // [b * C * hq * (topk-1), d]  normalised partial outputs
   float* part_lse;      // [b * C * hq * (topk-1)]     their log2-sum-exp2
   int32_t* tile_start;  // [b * hkv * n + 1]           tile prefix of one pass

@@ -64,13 +64,14 @@ moba::Dims make_dims(const moba_shape_t* s) {
 size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct AttnLayout {
-  size_t part_o, part_lse, tile_start, total;
+  size_t status, part_o, part_lse, tile_start, total;
 };
 AttnLayout attn_layout(const moba_shape_t* s) {
   const size_t KH = s->topk - 1;
   const size_t entries = (size_t)s->batch * chunk_of(s) * s->hq * KH;
   AttnLayout L;
-  L.part_o = 0;
+  L.status = 0;
+  L.part_o = 256;
   L.part_lse = L.part_o + align_up(entries * s->head_dim * sizeof(float));
   L.tile_start = L.part_lse + align_up(entries * sizeof(float));
   L.total = L.tile_start + align_up(((size_t)s->batch * s->hkv * nblocks(s) + 1) * sizeof(int32_t));
@@ -191,7 +192,8 @@ MOBA_API moba_status_t moba_attn_fwd(const moba_shape_t* s, const void* q, const
   if (ws_bytes < moba_attn_workspace_size(s)) return MOBA_ERR_WORKSPACE;
   AttnLayout L = attn_layout(s);
   char* base = static_cast<char*>(ws);
-  moba::AttnWs a{reinterpret_cast<float*>(base + L.part_o), reinterpret_cast<float*>(base + L.part_lse),
+  moba::AttnWs a{reinterpret_cast<int*>(base + L.status), reinterpret_cast<float*>(base + L.part_o),
+                 reinterpret_cast<float*>(base + L.part_lse),
                  reinterpret_cast<int32_t*>(base + L.tile_start)};
   int launches = 0;
   cudaError_t e = moba::launch_attn(make_dims(s), s->dtype, q, k, v, sel, offsets, rows, out, lse, a,
