@@ -154,7 +154,11 @@ MOBA_API moba_status_t moba_block_meanpool(const moba_shape_t* shape, const void
  *            r = (b * seqlen + t) * hq + h (the row of q viewed as
  *            [batch*seqlen*hq, head_dim]); within a group the order is
  *            unspecified.
- *   ws       >= moba_gate_workspace_size bytes of device scratch. */
+ *   ws       >= moba_gate_workspace_size bytes of device scratch.  After the
+ *            call completes on the stream, the int32 at byte offset
+ *            moba_gate_workspace_size - 256 holds 0, or MOBA_ERR_TIMEOUT if a
+ *            bounded device-side wait of the tensor-core scoring kernel expired
+ *            (the results are then invalid). */
 MOBA_API moba_status_t moba_gate_topk(const moba_shape_t* shape, const void* q, const float* meank,
                                       int32_t* sel, int32_t* offsets, int32_t* rows, void* ws,
                                       size_t ws_bytes, moba_stream_t stream);
@@ -168,7 +172,11 @@ MOBA_API moba_status_t moba_gate_topk(const moba_shape_t* shape, const void* q, 
  *   sel, offsets, rows outputs of moba_gate_topk             (read)
  *   out   [batch, seqlen, hq, head_dim] dtype                (written)
  *   lse   [batch, hq, seqlen] fp32, natural log, or NULL     (written)
- *   ws    >= moba_attn_workspace_size bytes of device scratch. */
+ *   ws    >= moba_attn_workspace_size bytes of device scratch.  After the call
+ *         completes on the stream, the first int32 of ws holds 0, or
+ *         MOBA_ERR_TIMEOUT if a bounded device-side wait of a tensor-core
+ *         kernel expired (out is then invalid).  Every wait in these kernels is
+ *         bounded (2 s), so a fault in the pipeline cannot hang the GPU. */
 MOBA_API moba_status_t moba_attn_fwd(const moba_shape_t* shape, const void* q, const void* k,
                                      const void* v, const int32_t* sel, const int32_t* offsets,
                                      const int32_t* rows, void* out, float* lse, void* ws,
@@ -185,6 +193,13 @@ MOBA_API int moba_last_cuda_error(void);
 /* Number of kernel launches the last moba_* call on this thread enqueued. */
 MOBA_API int moba_last_launch_count(void);
 
+/* Self-test of the failure path shared by the tensor-core kernels (the paper
+ * has no counterpart): one kernel waits, with the same bounded wait, on an
+ * mbarrier that nothing arrives at.  After about 2 s it gives up and writes
+ * MOBA_ERR_TIMEOUT to *status (a device int32); the context stays usable.
+ * Nothing faults, traps or hangs. */
+MOBA_API moba_status_t moba_selftest_bounded_wait(int* status, moba_stream_t stream);
+
 /* ---- gate without caller-provided scratch ----------------------------- */
 
 /* Groups (offsets entries minus one) the allocation-free gate can index. */
@@ -198,7 +213,7 @@ MOBA_API int moba_last_launch_count(void);
  *
  * Same arguments, results and layouts as moba_gate_topk, minus ws/ws_bytes.
  * The scratch (two int32 counters per group) lives in a fixed array inside
- * the library: 2 * MOBA_GATE_NOALLOC_MAX_GROUPS int32 (4 MiB), held on every
+ * the library: 2 * MOBA_GATE_NOALLOC_MAX_GROUPS + 64 int32 (4 MiB), held on every
  * GPU that loads the library until the process exits.  Shapes with more than
  * MOBA_GATE_NOALLOC_MAX_GROUPS groups (moba_offsets_elems - 1) are rejected
  * with MOBA_ERR_UNSUPPORTED before anything is enqueued.

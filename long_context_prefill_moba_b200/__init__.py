@@ -45,7 +45,7 @@ EXPORTED_SYMBOLS = [
     "moba_meank_elems", "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems",
     "moba_gate_workspace_size", "moba_attn_workspace_size", "moba_block_meanpool",
     "moba_gate_topk", "moba_attn_fwd", "moba_status_string", "moba_last_cuda_error",
-    "moba_last_launch_count", "moba_gate_topk_noalloc",
+    "moba_last_launch_count", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait",
 ]
 
 
@@ -99,6 +99,8 @@ def load_library(path: str = LIB_PATH):
     L.moba_gate_topk.restype = st
     L.moba_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moba_attn_fwd.restype = st
+    L.moba_selftest_bounded_wait.argtypes = [vp, vp]
+    L.moba_selftest_bounded_wait.restype = st
     L.moba_gate_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
     L.moba_gate_topk_noalloc.restype = st
     L.moba_status_string.argtypes = [st]
@@ -179,6 +181,11 @@ def moba_gate_topk_noalloc(shape, q, meank, sel, offsets, rows, stream=None):
            "moba_gate_topk_noalloc")
 
 
+def moba_selftest_bounded_wait(status, stream=None):
+    """Run the bounded-wait self-test kernel; `status` is a 1-element int32 CUDA tensor."""
+    _check(lib().moba_selftest_bounded_wait(_ptr(status), _stream(stream)), "moba_selftest_bounded_wait")
+
+
 def moba_attn_fwd(shape, q, k, v, sel, offsets, rows, out, lse, ws, stream=None):
     _check(lib().moba_attn_fwd(_s(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(offsets),
                                _ptr(rows), _ptr(out), _ptr(lse), _ptr(ws),
@@ -224,6 +231,14 @@ class MobaLayer:
         n += moba_last_launch_count()
         self.launches = n
         return out
+
+    def device_status(self):
+        """(gate, attention) device status words of the last forward (synchronises):
+        0, or MOBA_ERR_TIMEOUT (6) if a bounded wait in a tensor-core kernel expired."""
+        torch.cuda.synchronize(self.device)
+        g = self.gate_ws[-256:-252].view(torch.int32).item()
+        a = self.attn_ws[:4].view(torch.int32).item()
+        return g, a
 
     def sel_view(self):
         s = self.shape

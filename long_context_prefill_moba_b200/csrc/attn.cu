@@ -16,6 +16,9 @@ cudaError_t launch_attn_mma_cur(const Dims& dm, const void* q, const void* k, co
 cudaError_t launch_attn_tc_hist(const Dims& dm, const void* q, const void* k, const void* v,
                                 const int32_t* sel, const int32_t* offsets, const int32_t* rows,
                                 const AttnWs& ws, int ch, int64_t grid, cudaStream_t stream);
+cudaError_t launch_attn_tc_cur(const Dims& dm, const void* q, const void* k, const void* v,
+                               const AttnWs& ws, void* out, float* lse, int ch,
+                               cudaStream_t stream);
 int attn_tc_rows_per_tile();
 cudaError_t launch_attn_f32_hist(const Dims& dm, const void* q, const void* k, const void* v,
                                  const int32_t* sel, const int32_t* offsets, const int32_t* rows,
@@ -43,7 +46,7 @@ cudaError_t launch_attn(const Dims& dm, int dtype, const void* q, const void* k,
   const int ngroups = dm.batch * dm.hkv * dm.n;
   cudaError_t e = cudaMemsetAsync(ws.status, 0, sizeof(int), stream);
   if (e != cudaSuccess) return e;
-  // bf16 with head_dim 128: tensor-core (tcgen05) kernel for the historical blocks
+  // bf16 with head_dim 128: tensor-core (tcgen05) kernels for both attention steps
   const bool tc = dtype == MOBA_BF16 && dm.d == 128;
   const int tm = tc ? attn_tc_rows_per_tile() : 64;
   for (int ch = 0; ch < dm.nchunks; ++ch) {
@@ -67,8 +70,9 @@ cudaError_t launch_attn(const Dims& dm, int dtype, const void* q, const void* k,
       ++*launches;
       if (e != cudaSuccess) return e;
     }
-    e = dtype == MOBA_BF16 ? launch_attn_mma_cur(dm, q, k, v, ws, out, lse, ch, stream)
-                           : launch_attn_f32_cur(dm, q, k, v, ws, out, lse, ch, stream);
+    e = tc ? launch_attn_tc_cur(dm, q, k, v, ws, out, lse, ch, stream)
+           : dtype == MOBA_BF16 ? launch_attn_mma_cur(dm, q, k, v, ws, out, lse, ch, stream)
+                                : launch_attn_f32_cur(dm, q, k, v, ws, out, lse, ch, stream);
     ++*launches;
     if (e != cudaSuccess) return e;
   }

@@ -1,14 +1,24 @@
-// K3a on 5th-generation tensor cores (tcgen05 + TMEM + TMA): attention of the
-// grouped queries over one earlier ("historical") block, no mask.
+// K3 on 5th-generation tensor cores (tcgen05 + TMEM + TMA): the two attention
+// steps of MoBA for bf16, head_dim 128.
 //
 // "MoBA: Mixture of Block Attention for Long-Context LLMs", paper-graph summary
-// §3 "The Core MoBA Attention Equation" and Implementation, Algorithm 1 Step 3:
-// the queries that routed to a block are gathered so that the block's keys and
-// values are loaded once for all of them; the per-row partial results are
-// merged later with the current-block part (Step 4).
+// §3 "The Core MoBA Attention Equation" (Softmax(q K[I]^T) V[I]), "Causality
+// Enforcement" mechanism 2 (causal mask inside the current block) and the
+// Implementation section, Algorithm 1 Step 3 (historical blocks without a
+// mask, the queries that routed to a block gathered so the block's keys and
+// values are loaded once for all of them; the current block causal) and Step 4
+// (online-softmax merge of the partial results).
 //
-// One CTA = one work tile of up to 256 query rows of one (b, kv head g, block j)
-// group, as two 128-row tiles Q0 / Q1 (TMEM lanes = rows).  Roles:
+// Two modes of one kernel template:
+//   kHist  one CTA = up to 256 query rows of one (b, kv head g, earlier block j)
+//          group (taken from the gate's `rows` list), all B keys of block j,
+//          no mask; writes each row's normalised partial (o, log2-sum-exp2).
+//   kCur   one CTA = 128 consecutive tokens of two query heads of one kv group
+//          (one head when the group size is odd and this is the last head);
+//          keys from the start of the first token's block up to the last
+//          token, causal inside each token's own block; the epilogue merges the
+//          row's historical partials and writes out (and lse).
+// The 256 rows are two 128-row tiles Q0 / Q1 (TMEM lanes = rows).  Roles:
 //   warps 0-3  softmax for Q0        warps 4-7  softmax for Q1
 //   warp 8     TMA producer of K/V tiles (and TMEM allocation)
 //   warp 9     single-thread tcgen05.mma issuer      warps 10-11 idle
@@ -40,12 +50,14 @@ namespace {
 
 using namespace sm100;
 
+constexpr int kHist = 0, kCur = 1;
+
 constexpr int kD = 128;
 constexpr int kQT = 128;                 // rows per Q tile
 constexpr int kBK = 128;                 // keys per K/V tile
 constexpr int kRowsPerCta = 2 * kQT;
 constexpr int kThreads = 384;
-constexpr int kLaunchRegs = 168;     // registers per thread at launch (ptxas, 384 threads, 1 CTA/SM)
+constexpr int kLaunchRegs = 168;         // registers per thread at launch (ptxas, 384 threads, 1 CTA/SM)
 constexpr int kSoftmaxRegs = 216;
 constexpr int kServiceRegs = 64;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kServiceRegs <= kThreads * kLaunchRegs,
@@ -57,6 +69,17 @@ constexpr uint32_t kOffK = 2 * kTile;    // stages at +0, +kTile
 constexpr uint32_t kOffV = 4 * kTile;
 constexpr uint32_t kSmemBytes = 6 * kTile + 1024;
 constexpr float kRescaleThreshold = 8.f; // log2 units: rescale O only when the max grows by > 2^8
+// Exponentials of pairs c with (c % kPolyPeriod) == kPolyPeriod - 1 run on the
+// FMA pipe (exp2_poly) instead of MUFU; 0 = never (measured fastest on B200
+// for this kernel, whose softmax is not MUFU-throughput bound).
+#ifndef MOBA_POLY_PERIOD
+#define MOBA_POLY_PERIOD 0
+#endif
+constexpr int kPolyPeriod = MOBA_POLY_PERIOD;
+// MUFU exponential: 1 = ex2.approx.ftz.f32 directly, 0 = exp2f
+#ifndef MOBA_EX2_DIRECT
+#define MOBA_EX2_DIRECT 1
+#endif
 
 struct Ctl {
   uint64_t q_full[2], k_full[2], v_full[2], k_free[2], v_free[2], s_full[2], p_full[2], o_full[2];
@@ -66,34 +89,74 @@ struct Ctl {
 };
 
 MOBA_DEV uint32_t bar(const uint64_t* b) { return smem_u32(b); }
+MOBA_DEV float ex2(float x) { return MOBA_EX2_DIRECT ? ex2_approx(x) : exp2f(x); }
 
-__global__ void __launch_bounds__(kThreads, 1) attn_hist_tc_kernel(
+struct Tile {
+  int b, g, nq;
+  int key0;        // sequence position of key tile 0
+  int nkt;         // key tiles
+  int j;           // kHist: the block
+  int r0, cnt;     // kHist: rows[r0 .. r0 + cnt)
+  int h0, t_first, t_last;   // kCur
+};
+
+template <int MODE>
+MOBA_DEV bool decode_tile(Tile& w, const int32_t* tile_start, const int32_t* offsets, const Dims& dm,
+                          int ch) {
+  const int t0 = ch * dm.chunk;
+  if (MODE == kHist) {
+    const int ngroups = dm.batch * dm.hkv * dm.n;
+    const int tile = blockIdx.x;
+    if (tile >= tile_start[ngroups]) return false;
+    int lo = 0, hi = ngroups - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    w.j = lo % dm.n;
+    w.g = (lo / dm.n) % dm.hkv;
+    w.b = lo / (dm.n * dm.hkv);
+    const size_t goff = (size_t)ch * ngroups + lo;
+    w.r0 = offsets[goff] + (tile - tile_start[lo]) * kRowsPerCta;
+    w.cnt = min(kRowsPerCta, offsets[goff + 1] - w.r0);
+    w.nq = w.cnt > kQT ? 2 : 1;
+    w.key0 = w.j * dm.B;
+    w.nkt = (dm.B + kBK - 1) / kBK;
+  } else {
+    const int t_end = min(dm.N, t0 + dm.chunk);
+    const int ntile = (t_end - t0 + kQT - 1) / kQT;
+    const int pairs = (dm.G + 1) / 2;
+    int idx = blockIdx.x;
+    const int tau = idx % ntile; idx /= ntile;
+    const int p = idx % pairs; idx /= pairs;
+    w.g = idx % dm.hkv;
+    w.b = idx / dm.hkv;
+    if (w.b >= dm.batch) return false;
+    w.h0 = w.g * dm.G + 2 * p;
+    w.nq = (2 * p + 1 < dm.G) ? 2 : 1;
+    w.t_first = t0 + tau * kQT;
+    w.t_last = min(t_end, w.t_first + kQT) - 1;
+    w.key0 = (w.t_first / dm.B) * dm.B;
+    w.nkt = (w.t_last - w.key0) / kBK + 1;
+  }
+  return true;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ sel,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ rows,
     const int32_t* __restrict__ tile_start, float* __restrict__ part_o,
-    float* __restrict__ part_lse, int* __restrict__ status, Dims dm, int ch) {
+    float* __restrict__ part_lse, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+    int* __restrict__ status, Dims dm, int ch) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ Ctl ctl;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
 
-  const int ngroups = dm.batch * dm.hkv * dm.n;
-  const int tile = blockIdx.x;
-  if (tile >= tile_start[ngroups]) return;
-  int lo = 0, hi = ngroups - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
-  }
-  const int grp = lo;
-  const int j = grp % dm.n;
-  const int g = (grp / dm.n) % dm.hkv;
-  const int b = grp / (dm.n * dm.hkv);
-  const size_t goff = (size_t)ch * ngroups + grp;
-  const int r0 = offsets[goff] + (tile - tile_start[grp]) * kRowsPerCta;
-  const int cnt = min(kRowsPerCta, offsets[goff + 1] - r0);
-  const int nq = cnt > kQT ? 2 : 1;
-  const int nkt = (dm.B + kBK - 1) / kBK;
+  Tile wk;
+  if (!decode_tile<MODE>(wk, tile_start, offsets, dm, ch)) return;
+  const int b = wk.b, g = wk.g, nq = wk.nq, nkt = wk.nkt;
   const int KH = dm.topk - 1;
   const int t0 = ch * dm.chunk;
 
@@ -132,9 +195,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_hist_tc_kernel(
     const int w = warp >> 2;
     if (w < nq) {
       const int rho = tid & 127;
-      const int row_i = w * kQT + rho;
-      const bool valid = row_i < cnt;
-      const int r = valid ? rows[r0 + row_i] : 0;
+      bool valid;
+      int r, t, h;
+      if (MODE == kHist) {
+        const int row_i = w * kQT + rho;
+        valid = row_i < wk.cnt;
+        r = valid ? rows[wk.r0 + row_i] : 0;
+        h = r % dm.hq;
+        t = (r / dm.hq) % dm.N;
+      } else {
+        t = wk.t_first + rho;
+        valid = t <= wk.t_last;
+        h = wk.h0 + w;
+        r = valid ? (b * dm.N + t) * dm.hq + h : 0;
+      }
       const uint32_t qs = base + kOffQ + w * kTile;
       const __nv_bfloat16* src = q + (size_t)r * kD;
 #pragma unroll
@@ -144,13 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_hist_tc_kernel(
       cp_async_wait<0>();
       fence_proxy_async_smem();
       mbar_arrive(bar(&ctl.q_full[w]));
-      size_t pidx = 0;
-      if (valid) {
-        const int h = r % dm.hq;
-        const int t = (r / dm.hq) % dm.N;
-        const int slot = slot_of(sel + (size_t)r * dm.topk, dm.topk, j);
-        pidx = (size_t)((b * dm.chunk + (t - t0)) * dm.hq + h) * KH + slot;
-      }
+      // causal window of this row in kCur: keys [lo_t, t]
+      const int lo_t = (t / dm.B) * dm.B;
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       const uint32_t tS = tb + (w ? 128u : 0u) + lane_off;
       const uint32_t tO = tb + (w ? 384u : 256u) + lane_off;
@@ -167,15 +236,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_hist_tc_kernel(
         tmem_ld32(tS + 64, sr + 64);
         tmem_ld32(tS + 96, sr + 96);
         tmem_wait_ld();
-        const int kvalid = dm.B - i * kBK;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float x = __uint_as_float(sr[c]);
-          if (c >= kvalid) x = -INFINITY;
-          sr[c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+        // keys of this tile valid for this row: positions [vlo, vhi] relative to the tile
+        const int u0 = wk.key0 + i * kBK;
+        int vlo, vhi;
+        if (MODE == kHist) {
+          vlo = 0;
+          vhi = dm.B - i * kBK - 1;
+        } else {
+          vlo = lo_t - u0;
+          vhi = t - u0;
         }
+        if (!(vlo <= 0 && vhi >= kBK - 1)) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c < vlo || c > vhi) sr[c] = __float_as_uint(-INFINITY);
+        }
+        // row max: four independent chains of three-input maxima, then a tree
+        float mx4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1]));
+#pragma unroll
+        for (int c = 8; c < 128; c += 8)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            mx4[u] = max3(mx4[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         const float mxs = mx * sl2;
         const bool need = mxs > m_used + kRescaleThreshold;
         if (i > 0 && __any_sync(0xffffffffu, need)) {
@@ -195,16 +280,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_hist_tc_kernel(
           l *= exp2f(m_used - mxs);
           m_used = mxs;
         }
-        float rs = 0.f;
+        // a row with no valid key yet keeps m_used = -inf: use 0 as the base (p = 0)
+        const float mb = m_used == -INFINITY ? 0.f : m_used;
+        // x = s * scale * log2(e) - base and the row sum run as packed pairs
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), nmbx2 = f2_pack(-mb, -mb);
+        uint64_t rs4[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = exp2f(fmaf(__uint_as_float(sr[2 * c]), sl2, -m_used));
-          const float p1 = exp2f(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m_used));
-          rs += p0 + p1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2, nmbx2),
+                    x0, x1);
+          const bool poly = kPolyPeriod > 0 && (c % (kPolyPeriod > 0 ? kPolyPeriod : 1)) == kPolyPeriod - 1;
+          const float p0 = poly ? exp2_poly(x0) : ex2(x0);
+          const float p1 = poly ? exp2_poly(x1) : ex2(x1);
+          rs4[c & 3] = f2_add(rs4[c & 3], f2_pack(p0, p1));
           pk[c] = pack_bf16x2(p0, p1);
         }
-        l += rs;
+        {
+          float a0, a1;
+          f2_unpack(f2_add(f2_add(rs4[0], rs4[1]), f2_add(rs4[2], rs4[3])), a0, a1);
+          l += a0 + a1;
+        }
         tmem_st32(tS + 0, pk);
         tmem_st32(tS + 32, pk + 32);
         tmem_wait_st();
@@ -214,22 +311,98 @@ __global__ void __launch_bounds__(kThreads, 1) attn_hist_tc_kernel(
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.o_full[w]), 0, abort_flag));
       if (ok) {
         tc_fence_after();
-        const float inv = 1.f / l;
-        float* dst = part_o + pidx * kD;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + cc * 32, o);
-          tmem_wait_ld();
+        const float lse2 = m_used + log2f(l);
+        if (MODE == kHist) {
+          size_t pidx = 0;
           if (valid) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(dst + cc * 32 + e) =
-                  make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                              __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            const int slot = slot_of(sel + (size_t)r * dm.topk, dm.topk, wk.j);
+            pidx = (size_t)((b * dm.chunk + (t - t0)) * dm.hq + h) * KH + slot;
           }
+          const float inv = 1.f / l;
+          // partials are kept in bf16 (the merge is done in fp32; the
+          // rounding, 2^-9 relative of a normalised output, stays far below
+          // the output tolerance) to halve their HBM traffic
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(part_o) + pidx * kD;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_wait_ld();
+            if (valid) {
+              uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+              for (int e8 = 0; e8 < 4; ++e8)
+                d4[e8] = make_uint4(
+                    pack_bf16x2(__uint_as_float(o[8 * e8 + 0]) * inv, __uint_as_float(o[8 * e8 + 1]) * inv),
+                    pack_bf16x2(__uint_as_float(o[8 * e8 + 2]) * inv, __uint_as_float(o[8 * e8 + 3]) * inv),
+                    pack_bf16x2(__uint_as_float(o[8 * e8 + 4]) * inv, __uint_as_float(o[8 * e8 + 5]) * inv),
+                    pack_bf16x2(__uint_as_float(o[8 * e8 + 6]) * inv, __uint_as_float(o[8 * e8 + 7]) * inv));
+            }
+          }
+          if (valid) part_lse[pidx] = lse2;
+        } else {
+          // merge with the historical partials of the row (Algorithm 1 Step 4)
+          const int nh = valid ? min(KH, t / dm.B) : 0;
+          const size_t pbase = (size_t)((b * dm.chunk + (t - t0)) * dm.hq + h) * KH;
+          float M = lse2;
+          for (int s = 0; s < nh; ++s) M = fmaxf(M, part_lse[pbase + s]);
+          const float wc = exp2f(lse2 - M);
+          float W = wc;
+          for (int s = 0; s < nh; ++s) W += exp2f(part_lse[pbase + s] - M);
+          const float iw = 1.f / W;
+          const float fc = wc / l * iw;
+          __nv_bfloat16* dst = out + (size_t)r * kD;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_wait_ld();
+            if (valid) {
+              float acc[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(o[e]) * fc;
+              const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(part_o);
+              // four slots per round so 16 loads are in flight
+              for (int s0 = 0; s0 < nh; s0 += 4) {
+                uint4 x[4][4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const uint4* src4 =
+                      reinterpret_cast<const uint4*>(pb + (pbase + s0 + u) * kD + cc * 32);
+#pragma unroll
+                  for (int e8 = 0; e8 < 4; ++e8)
+                    x[u][e8] = (s0 + u < nh) ? __ldg(src4 + e8) : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  if (s0 + u < nh) {
+                    const float ws = exp2f(part_lse[pbase + s0 + u] - M) * iw;
+#pragma unroll
+                    for (int e8 = 0; e8 < 4; ++e8) {
+                      const uint32_t w4[4] = {x[u][e8].x, x[u][e8].y, x[u][e8].z, x[u][e8].w};
+#pragma unroll
+                      for (int h2 = 0; h2 < 4; ++h2) {
+                        const float2 f2 =
+                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[h2]));
+                        acc[8 * e8 + 2 * h2] = fmaf(ws, f2.x, acc[8 * e8 + 2 * h2]);
+                        acc[8 * e8 + 2 * h2 + 1] = fmaf(ws, f2.y, acc[8 * e8 + 2 * h2 + 1]);
+                      }
+                    }
+                  }
+                }
+              }
+              uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+              for (int e8 = 0; e8 < 4; ++e8)
+                d4[e8] = make_uint4(pack_bf16x2(acc[8 * e8 + 0], acc[8 * e8 + 1]),
+                                    pack_bf16x2(acc[8 * e8 + 2], acc[8 * e8 + 3]),
+                                    pack_bf16x2(acc[8 * e8 + 4], acc[8 * e8 + 5]),
+                                    pack_bf16x2(acc[8 * e8 + 6], acc[8 * e8 + 7]));
+            }
+          }
+          if (valid && lse != nullptr)
+            lse[((size_t)b * dm.hq + h) * dm.N + t] = (M + log2f(W)) * kLn2;
         }
-        if (valid) part_lse[pidx] = m_used + log2f(l);
       }
     }
   } else if (warp == 8) {
@@ -237,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_hist_tc_kernel(
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const int y0 = b * dm.N + j * dm.B;
+      const int y0 = b * dm.N + wk.key0;
       const int x0 = g * kD;
       int issued_k = 0, issued_v = 0;
       for (int i = 0; i < nkt; ++i) {
@@ -368,33 +541,55 @@ bool make_kv_map(CUtensorMap* map, const void* base, const Dims& dm) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// the setmaxnreg split is only safe if the kernel really launches with kLaunchRegs
+template <int MODE>
+cudaError_t check_regs() {
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_tc_kernel<MODE>);
+    if (e != cudaSuccess) return e;
+    regs = fa.numRegs;
+  }
+  return regs >= kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+template <int MODE>
+cudaError_t launch_tc(const Dims& dm, const void* q, const void* k, const void* v,
+                      const int32_t* sel, const int32_t* offsets, const int32_t* rows,
+                      const AttnWs& ws, void* out, float* lse, int ch, int64_t grid,
+                      cudaStream_t stream) {
+  CUtensorMap mk, mv;
+  if (!make_kv_map(&mk, k, dm) || !make_kv_map(&mv, v, dm)) return cudaErrorInvalidValue;
+  cudaError_t e = check_regs<MODE>();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kSmemBytes);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, stream>>>(
+      (const __nv_bfloat16*)q, mk, mv, sel, offsets, rows, ws.tile_start, ws.part_o, ws.part_lse,
+      (__nv_bfloat16*)out, lse, ws.status, dm, ch);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
-constexpr int kTcRowsPerTile = kRowsPerCta;
+int attn_tc_rows_per_tile() { return kRowsPerCta; }
 
 cudaError_t launch_attn_tc_hist(const Dims& dm, const void* q, const void* k, const void* v,
                                 const int32_t* sel, const int32_t* offsets, const int32_t* rows,
                                 const AttnWs& ws, int ch, int64_t grid, cudaStream_t stream) {
-  CUtensorMap mk, mv;
-  if (!make_kv_map(&mk, k, dm) || !make_kv_map(&mv, v, dm)) return cudaErrorInvalidValue;
-  // the setmaxnreg split is only safe if the kernel really launches with kLaunchRegs
-  static int launch_regs = -1;
-  if (launch_regs < 0) {
-    cudaFuncAttributes fa;
-    cudaError_t ea = cudaFuncGetAttributes(&fa, attn_hist_tc_kernel);
-    if (ea != cudaSuccess) return ea;
-    launch_regs = fa.numRegs;
-  }
-  if (launch_regs < kLaunchRegs) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(attn_hist_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmemBytes);
-  if (e != cudaSuccess) return e;
-  attn_hist_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
-      (const __nv_bfloat16*)q, mk, mv, sel, offsets, rows, ws.tile_start, ws.part_o, ws.part_lse,
-      ws.status, dm, ch);
-  return cudaGetLastError();
+  return launch_tc<kHist>(dm, q, k, v, sel, offsets, rows, ws, nullptr, nullptr, ch, grid, stream);
 }
 
-int attn_tc_rows_per_tile() { return kTcRowsPerTile; }
+cudaError_t launch_attn_tc_cur(const Dims& dm, const void* q, const void* k, const void* v,
+                               const AttnWs& ws, void* out, float* lse, int ch,
+                               cudaStream_t stream) {
+  const int t0 = ch * dm.chunk;
+  const int t_end = dm.N < t0 + dm.chunk ? dm.N : t0 + dm.chunk;
+  const int64_t ntile = (t_end - t0 + kQT - 1) / kQT;
+  const int64_t grid = ntile * ((dm.G + 1) / 2) * dm.hkv * dm.batch;
+  return launch_tc<kCur>(dm, q, k, v, nullptr, nullptr, nullptr, ws, out, lse, ch, grid, stream);
+}
 
 }  // namespace moba

@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/moba.h"
+#include "moba.h"
 
 #define MOBA_DEV __device__ __forceinline__
 

@@ -116,9 +116,10 @@ __global__ void __launch_bounds__(kRows) gate_select_kernel(const T* __restrict_
           }
         }
         kept = min(kept + 1, KH);
+        // threshold = smallest kept score; a predicated min keeps indices compile-time
+        thresh = INFINITY;
 #pragma unroll
-        for (int i = 0; i < MOBA_MAX_TOPK; ++i)
-          if (i == KH - 1) thresh = ts[i];
+        for (int i = 0; i < MOBA_MAX_TOPK; ++i) thresh = fminf(thresh, i < KH ? ts[i] : INFINITY);
       }
     }
   }
@@ -268,8 +269,13 @@ cudaError_t launch_gate(const Dims& dm, int dtype, const void* q, const float* m
   const int64_t L = (int64_t)dm.nchunks * dm.batch * dm.hkv * dm.n;
   cudaError_t e = cudaMemsetAsync(ws.counts, 0, sizeof(int32_t) * L * 2, stream);  // counts+cursors
   if (e != cudaSuccess) return e;
-  e = dtype == MOBA_BF16 ? launch_select<__nv_bfloat16>(dm, q, meank, sel, ws.counts, stream)
-                         : launch_select<float>(dm, q, meank, sel, ws.counts, stream);
+  if ((e = cudaMemsetAsync(ws.status, 0, sizeof(int), stream)) != cudaSuccess) return e;
+  if (gate_tc_supported(dm, dtype))
+    e = launch_gate_select_tc(dm, q, meank, sel, ws.counts, ws.status, stream);
+  else if (dtype == MOBA_BF16)
+    e = launch_select<__nv_bfloat16>(dm, q, meank, sel, ws.counts, stream);
+  else
+    e = launch_select<float>(dm, q, meank, sel, ws.counts, stream);
   ++*launches;
   if (e != cudaSuccess) return e;
   gate_scan_kernel<<<1, kScanThreads, 0, stream>>>(ws.counts, offsets, L);
@@ -296,7 +302,7 @@ cudaError_t launch_gate(const Dims& dm, int dtype, const void* q, const float* m
 namespace {
 
 constexpr int kNoAllocMaxDevices = 64;
-static __device__ __align__(256) int32_t g_gate_scratch[2 * MOBA_GATE_NOALLOC_MAX_GROUPS];
+static __device__ __align__(256) int32_t g_gate_scratch[2 * MOBA_GATE_NOALLOC_MAX_GROUPS + 64];
 
 std::mutex g_scratch_mu;
 int32_t* g_scratch_ptr[kNoAllocMaxDevices] = {};
@@ -330,7 +336,7 @@ cudaError_t launch_gate_noalloc(const Dims& dm, int dtype, const void* q, const 
   cudaError_t e = scratch_for_current_device(&scratch);
   if (e != cudaSuccess) return e;
   const int64_t L = (int64_t)dm.nchunks * dm.batch * dm.hkv * dm.n;
-  GateWs ws{scratch, scratch + L};   // counts, then cursors; launch_gate clears both
+  GateWs ws{scratch, scratch + L, scratch + 2 * L};   // counts, cursors, status; launch_gate clears them
   return launch_gate(dm, dtype, q, meank, sel, offsets, rows, ws, stream, launches);
 }
 

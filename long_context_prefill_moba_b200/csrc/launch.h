@@ -21,7 +21,13 @@ cudaError_t launch_meanpool(const Dims& dm, int dtype, const void* k, float* mea
 struct GateWs {
   int32_t* counts;   // [ngroups] rows per (chunk, b, g, j)
   int32_t* cursors;  // [ngroups] scatter cursors
+  int* status;       // device status word: 0, or MOBA_ERR_TIMEOUT after a bounded wait expired
 };
+
+// tensor-core scores + selection (bf16, head_dim 128, at most 256 blocks)
+bool gate_tc_supported(const Dims& dm, int dtype);
+cudaError_t launch_gate_select_tc(const Dims& dm, const void* q, const float* meank, int32_t* sel,
+                                  int32_t* counts, int* status, cudaStream_t stream);
 cudaError_t launch_gate(const Dims& dm, int dtype, const void* q, const float* meank, int32_t* sel,
                         int32_t* offsets, int32_t* rows, GateWs ws, cudaStream_t stream,
                         int* launches);
@@ -41,5 +47,8 @@ struct AttnWs {
 cudaError_t launch_attn(const Dims& dm, int dtype, const void* q, const void* k, const void* v,
                         const int32_t* sel, const int32_t* offsets, const int32_t* rows, void* out,
                         float* lse, AttnWs ws, cudaStream_t stream, int* launches);
+
+// a kernel whose only wait can never complete: it must time out (status word)
+cudaError_t launch_bounded_wait_selftest(int* status, cudaStream_t stream);
 
 }  // namespace moba

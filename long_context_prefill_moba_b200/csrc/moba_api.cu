@@ -133,7 +133,7 @@ MOBA_API int64_t moba_rows_elems(const moba_shape_t* s) {
 }
 MOBA_API size_t moba_gate_workspace_size(const moba_shape_t* s) {
   if (moba_check_shape(s) != MOBA_OK) return 0;
-  return align_up(2 * (size_t)ngroups_total(s) * sizeof(int32_t));
+  return align_up(2 * (size_t)ngroups_total(s) * sizeof(int32_t)) + 256;   // counters + status word
 }
 MOBA_API size_t moba_attn_workspace_size(const moba_shape_t* s) {
   if (moba_check_shape(s) != MOBA_OK) return 0;
@@ -167,7 +167,8 @@ MOBA_API moba_status_t moba_gate_topk(const moba_shape_t* s, const void* q, cons
     return MOBA_ERR_INVALID_ARG;
   if (ws_bytes < moba_gate_workspace_size(s)) return MOBA_ERR_WORKSPACE;
   const int64_t L = ngroups_total(s);
-  moba::GateWs g{static_cast<int32_t*>(ws), static_cast<int32_t*>(ws) + L};
+  moba::GateWs g{static_cast<int32_t*>(ws), static_cast<int32_t*>(ws) + L,
+                 reinterpret_cast<int*>(static_cast<char*>(ws) + align_up(2 * (size_t)L * sizeof(int32_t)))};
   int launches = 0;
   cudaError_t e = moba::launch_gate(make_dims(s), s->dtype, q, meank, sel, offsets, rows, g,
                                     (cudaStream_t)stream, &launches);
@@ -231,6 +232,12 @@ MOBA_API const char* moba_status_string(moba_status_t st) {
     case MOBA_ERR_TIMEOUT: return "MOBA_ERR_TIMEOUT: device wait timed out";
   }
   return "unknown moba_status_t";
+}
+
+MOBA_API moba_status_t moba_selftest_bounded_wait(int* status, moba_stream_t stream) {
+  g_last_launches = 0;
+  if (status == nullptr || !aligned4(status)) return MOBA_ERR_INVALID_ARG;
+  return finish(moba::launch_bounded_wait_selftest(status, (cudaStream_t)stream), 1);
 }
 
 MOBA_API int moba_last_cuda_error(void) { return g_last_cuda_error; }

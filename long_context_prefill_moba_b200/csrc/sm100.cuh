@@ -152,8 +152,66 @@ MOBA_DEV void tmem_st32(uint32_t taddr, const uint32_t* r) {
       "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+MOBA_DEV void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 MOBA_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 MOBA_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// Packed fp32 pair arithmetic (one instruction for two lanes of work) and the
+// three-input max, used to cut the softmax instruction count.
+MOBA_DEV uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+MOBA_DEV void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+MOBA_DEV uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+MOBA_DEV uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+MOBA_DEV float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the special-function unit: the PTX approximate base-2 exponential
+// (flush-to-zero; arguments here are <= 8 and results below 2^-126 do not
+// matter for a softmax)
+MOBA_DEV float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x on the FMA pipe (offloads the special-function unit in the softmax).
+// x = n + f with n = rint(x) (by the 1.5 * 2^23 rounding trick) and
+// f in [-0.5, 0.5]; 2^f is a degree-3 polynomial fitted in this project by
+// iteratively reweighted least squares on the relative error (max relative
+// error 7.5e-5, far below the 2^-9 rounding of the bf16 probabilities it
+// feeds); 2^n is added to the exponent field.  Inputs below -126 give ~1e-38.
+MOBA_DEV float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float r = x + 12582912.f;
+  const float f = x - (r - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.05517206f, f, 0.24261241f), f, 0.69326101f), f, 0.99992796f);
+  const int n = __float_as_int(r) - 0x4B400000;   // bits of 12582912.f
+  return __int_as_float(__float_as_int(p) + (n << 23));
+}
 
 // byte offset of the 16-byte chunk `c` (0..7) of row `r` inside a 128-byte
 // swizzled tile of 128-byte rows (atoms of 8 rows x 128 B, 1024-B aligned)

@@ -28,6 +28,7 @@ def run_gpu(cfg, query_chunk=0, with_lse=True):
     lse = torch.empty(cfg.batch, cfg.hq, cfg.seqlen, dtype=torch.float32, device=dev) if with_lse else None
     layer.forward(q, k, v, out, lse)
     torch.cuda.synchronize()
+    assert layer.device_status() == (0, 0)
     return dict(layer=layer, out=out, lse=lse, q=q, k=k, v=v)
 
 

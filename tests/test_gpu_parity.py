@@ -125,3 +125,16 @@ def test_10m_sampled(cuda_device):
     print("10m worst", worst)
     del res
     torch.cuda.empty_cache()
+
+
+def test_bounded_wait_times_out_and_context_survives(cuda_device):
+    """Failure detection on the GPU: a wait on a barrier that nothing arrives at
+    gives up after its limit with MOBA_ERR_TIMEOUT, and the context stays usable."""
+    import long_context_prefill_moba_b200 as M
+    status = torch.full((1,), -1, dtype=torch.int32, device=cuda_device)
+    M.moba_selftest_bounded_wait(status)
+    torch.cuda.synchronize()
+    assert status.item() == 6
+    cfg = EDGE["ragged_multipass"]
+    res = run_gpu(cfg, query_chunk=CHUNK["ragged_multipass"])
+    full_parity(cfg, res)

@@ -304,3 +304,27 @@ def test_algorithmic_pairs_brute_force(N, B, topk):
         sel, _ = O.select_blocks(np.arange(n, dtype=float), t, B, topk)
         total += len(O.key_positions(sel, t, B, N))
     assert O.algorithmic_pairs(2, N, 3, B, topk) == 2 * 3 * total
+
+
+# --------------------------------------------------------------------------
+# the FMA-pipe exponential used for part of the softmax (csrc/sm100.cuh,
+# exp2_poly): its fitted polynomial's relative error bound, checked in fp32
+# arithmetic against the exact 2^x over the range the softmax uses
+# --------------------------------------------------------------------------
+def test_exp2_polynomial_error_bound():
+    x = np.concatenate([np.linspace(-126.0, 8.0, 400001), -np.random.default_rng(0).random(100000) * 30])
+    x = x.astype(np.float32)
+    f32 = np.float32
+    xc = np.maximum(x, f32(-126.0))
+    r = (xc + f32(12582912.0)).astype(np.float32)
+    f = (xc - (r - f32(12582912.0))).astype(np.float32)
+    p = f32(0.05517206)
+    for cst in (0.24261241, 0.69326101, 0.99992796):
+        p = (p.astype(np.float64) * f + cst).astype(np.float32)       # fma: one rounding
+    n = r.view(np.int32) - np.int32(0x4B400000)
+    y = (p.view(np.int32) + (n << 23)).view(np.float32).astype(np.float64)
+    ref = np.exp2(xc.astype(np.float64))
+    normal = x >= -125.0
+    rel = np.abs(y[normal] - ref[normal]) / ref[normal]
+    assert rel.max() < 1e-4             # bf16 probabilities round at 2^-9 = 2e-3
+    assert np.all((y[~normal] >= 0) & (y[~normal] < 1e-37))   # clamped tail: negligible, never negative
