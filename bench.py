@@ -48,6 +48,27 @@ def attn_flops(cfg) -> float:
     return 4.0 * cfg.head_dim * algorithmic_pairs(cfg)
 
 
+def recorded_traffic(rows_per_layer: int):
+    """DRAM bytes of one attention step (moba_attn_fwd) from the committed ncu
+    capture (profiles/attn_traffic.json), scaled by the rows the gate routes
+    (the partial results and the gathered q rows dominate and grow with them).
+    None when the attention kernels changed since the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(p):
+        return None, "no capture"
+    with open(p) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "long_context_prefill_moba_b200", "csrc", "attn_tc.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if sha != d.get("kernel_source_sha256"):
+        return None, "kernel changed since the capture"
+    return d["dram_bytes_per_row"] * rows_per_layer, (
+        f"ncu capture of the {d['config']} layer ({d['dram_bytes_per_layer'] / 1e9:.2f} GB), "
+        f"scaled by routed rows")
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -122,13 +143,21 @@ def dist_setup():
     return world, rank, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Max of a per-rank timing over all ranks (the job's time is its slowest rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(per_rank_units: float, per_rank_ms: float, world: int, device: str = "cuda") -> float:
+    """Whole-job throughput: units of all ranks (every replica runs the same
+    work) divided by the slowest rank's time."""
+    ms = max_over_ranks(per_rank_ms, world, device)
+    return world * per_rank_units / (ms * 1e-3)
 
 
 def barrier(world: int):
@@ -302,14 +331,14 @@ def main():
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
-    ms = start.elapsed_time(end) / args.steps
-    ms = max_over_ranks(ms, world)
+    ms_rank = start.elapsed_time(end) / args.steps
     pool_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     gate_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
 
     flops = attn_flops(cfg)
-    value = world * flops / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(ms_rank, world)
+    value = job_throughput(flops, ms_rank, world) / 1e12
     peaks, peak_kind = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     attn_tf = flops / (attn_ms * 1e-3) / 1e12
@@ -318,6 +347,7 @@ def main():
     qbytes = cfg.batch * cfg.seqlen * cfg.hq * cfg.head_dim * esz
     pool_bytes = kbytes + layer.meank.numel() * 4
     gate_bytes = qbytes + layer.sel.numel() * 4 * 2 + layer.rows.numel() * 4
+    traffic, traffic_note = recorded_traffic(M.moba_rows_elems(sh))
 
     # end to end through the C ABI with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -337,8 +367,9 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
-        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e_rank = e0.elapsed_time(e1) / args.e2e_steps
+        e2e_ms = max_over_ranks(e2e_rank, world)
+        e2e = {"value": job_throughput(flops, e2e_rank, world) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 2 * kbytes + qbytes, "d2h_bytes_per_step": qbytes}
         del hq_, hk_, hv_, ho
 
@@ -356,7 +387,8 @@ def main():
             "kernels_ms": {"meanpool": pool_ms, "gate": gate_ms, "attn": attn_ms},
             "roofline": {"bound": "tensor", "kernel": "moba_attn_fwd (attention + merge)",
                          "achieved": attn_tf, "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
-                         "peak_kind": f"{peak_kind} bf16 sustained", "traffic": None},
+                         "peak_kind": f"{peak_kind} bf16 sustained", "traffic": traffic,
+                         "traffic_note": traffic_note},
             "hbm_kernels": {
                 "meanpool": {"achieved": pool_bytes / (pool_ms * 1e-3) / 1e9, "unit": "GB/s",
                              "peak": peaks["hbm_gbs"]},
