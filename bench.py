@@ -263,6 +263,72 @@ def config_of(cfg, args):
 
 
 # ---------------------------------------------------------------------------
+# Speed-up curve: MoBA layer vs dense causal attention at growing lengths
+# (the comparison of the paper's Figure 2a, on this GPU)
+# ---------------------------------------------------------------------------
+def speedup_curve(seqlens, reps=2):
+    """One JSON line per sequence length: the MoBA layer (mean-pool + gate +
+    attention through the C ABI) against dense causal attention on the same
+    q, k, v computed by torch's scaled_dot_product_attention (a library
+    FlashAttention-class kernel; cuDNN when available) and, where its index fits,
+    by this library itself with topk >= n (dense through the MoBA kernels)."""
+    import long_context_prefill_moba_b200 as M
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    M.load_library()
+    dev = torch.device("cuda", 0)
+    base = S.get_config("1m")
+    for N in seqlens:
+        cfg = base.replace(name=f"llama8b_{N // 1024}k", seqlen=N)
+        q, k, v = S.gen_q(cfg, dev), S.gen_k(cfg, dev), S.gen_v(cfg, dev)
+        out = torch.empty_like(q)
+
+        def timed(fn):
+            fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / reps
+
+        layer = M.MobaLayer.from_config(cfg, dev)
+        moba_ms = timed(lambda: layer.forward(q, k, v, out))
+        del layer
+        dense_self = None
+        dcfg = cfg.replace(topk=min(16, cfg.nblocks + 1))
+        dshape = M.make_shape(dcfg.batch, dcfg.seqlen, dcfg.hq, dcfg.hkv, dcfg.head_dim, dcfg.block,
+                              dcfg.topk, dcfg.dtype)
+        if dcfg.topk > dcfg.nblocks and M.moba_check_shape(dshape) == 0:
+            dl = M.MobaLayer.from_config(dcfg, dev)
+            dense_self = timed(lambda: dl.forward(q, k, v, out))
+            del dl
+        qt, kt, vt = (x.transpose(1, 2).contiguous() for x in (q, k, v))
+        backend = None
+        dense_ms = None
+        for be in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION):
+            try:
+                with sdpa_kernel([be]):
+                    dense_ms = timed(lambda: torch.nn.functional.scaled_dot_product_attention(
+                        qt, kt, vt, is_causal=True, scale=cfg.softmax_scale, enable_gqa=True))
+                backend = str(be).split(".")[-1]
+                break
+            except Exception:   # backend not available for this shape or build
+                continue
+        dense_flops = 4.0 * cfg.head_dim * cfg.batch * cfg.hq * N * (N + 1) / 2
+        print(json.dumps({
+            "mode": "speedup_curve", "seqlen": N, "hq": cfg.hq, "hkv": cfg.hkv, "block": cfg.block,
+            "topk": cfg.topk, "moba_ms": moba_ms, "moba_tflops": attn_flops(cfg) / moba_ms / 1e9,
+            "dense_ms": dense_ms, "dense_backend": backend,
+            "dense_tflops": None if dense_ms is None else dense_flops / dense_ms / 1e9,
+            "speedup_vs_dense": None if dense_ms is None else dense_ms / moba_ms,
+            "dense_via_moba_kernels_ms": dense_self}), flush=True)
+        del q, k, v, out, qt, kt, vt
+        torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 def main():
@@ -277,7 +343,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--speedup-curve", action="store_true",
+                    help="MoBA vs dense causal attention at growing lengths (one line per length)")
+    ap.add_argument("--curve-seqlens", default="32768,131072,262144,524288,1048576")
     args = ap.parse_args()
+    if args.speedup_curve:
+        speedup_curve([int(x) for x in args.curve_seqlens.split(",")])
+        return
     cfg = S.get_config(args.config)
 
     world, rank, local = dist_setup()

@@ -138,3 +138,31 @@ def test_bounded_wait_times_out_and_context_survives(cuda_device):
     cfg = EDGE["ragged_multipass"]
     res = run_gpu(cfg, query_chunk=CHUNK["ragged_multipass"])
     full_parity(cfg, res)
+
+
+MID = {
+    # several passes over a long sequence with GQA 4 and two batch entries (tensor-core paths)
+    "gqa4_b2_multipass": (S.get_config("1m").replace(batch=2, seqlen=20000, block=1024, topk=5),
+                          4096),
+    # a custom softmax scale and an odd block size
+    "scale_and_odd_block": (S.get_config("mqar").replace(batch=1, seqlen=3000, hq=8, hkv=4, block=320,
+                                                         topk=4, scale=0.05), 0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MID))
+def test_mid_size_sampled(cuda_device, name):
+    cfg, chunk = MID[name]
+    res = run_gpu(cfg, query_chunk=chunk)
+    worst = sampled_parity(cfg, res, sampled_rows(cfg, 48, seed=11))
+    print(name, "worst", worst)
+
+
+def test_convenience_forward_matches_layer(cuda_device):
+    import long_context_prefill_moba_b200 as M
+    cfg = EDGE["ragged_multipass"]
+    res = run_gpu(cfg)
+    out, lse = M.moba_forward(res["q"], res["k"], res["v"], cfg.block, cfg.topk, return_lse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out, res["out"])
+    assert torch.equal(lse, res["lse"])
