@@ -69,13 +69,23 @@ constexpr uint32_t kOffK = 2 * kTile;    // stages at +0, +kTile
 constexpr uint32_t kOffV = 4 * kTile;
 constexpr uint32_t kSmemBytes = 6 * kTile + 1024;
 constexpr float kRescaleThreshold = 8.f; // log2 units: rescale O only when the max grows by > 2^8
-// Exponentials of pairs c with (c % kPolyPeriod) == kPolyPeriod - 1 run on the
-// FMA pipe (exp2_poly) instead of MUFU; 0 = never (measured fastest on B200
-// for this kernel, whose softmax is not MUFU-throughput bound).
-#ifndef MOBA_POLY_PERIOD
-#define MOBA_POLY_PERIOD 0
+// A tile whose probabilities, taken against the row's current base, sum to at
+// most 2^15 (so none exceeds 2^15) is accepted without computing its row max.
+constexpr float kFastSumLimit = 32768.f;
+// Of every 8 pairs of exponentials, this many run on the FMA pipe
+// (exp2_poly2) and the rest on the special-function unit, whose 16 results
+// per clock per SM alone would take as long as the tile's two MMAs.
+#ifndef MOBA_POLY_OF8
+#define MOBA_POLY_OF8 0
 #endif
-constexpr int kPolyPeriod = MOBA_POLY_PERIOD;
+constexpr int kPolyOf8 = MOBA_POLY_OF8;
+static_assert(kPolyOf8 >= 0 && kPolyOf8 <= 8, "pairs per 8");
+// merge staging in the current-block epilogue: per softmax warp kMergeStages
+// slots of 32 rows x 256 bytes; the 8 warps' stages fill the Q/K/V buffers
+constexpr int kMergeStages = 3;
+constexpr uint32_t kMergeSlotBytes = 32 * kD * 2;
+constexpr uint32_t kMergeWarpBytes = kMergeStages * kMergeSlotBytes;
+static_assert(8 * kMergeWarpBytes <= 6 * kTile, "merge staging exceeds the tile buffers");
 // MUFU exponential: 1 = ex2.approx.ftz.f32 directly, 0 = exp2f
 #ifndef MOBA_EX2_DIRECT
 #define MOBA_EX2_DIRECT 1
@@ -226,11 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       const float sl2 = dm.scale_log2;
       float m_used = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int i = 0; i < nkt && ok; ++i) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.s_full[w]), i & 1, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t sr[128];
+      // S tile i into registers, keys outside the row's window set to -inf
+      auto load_s = [&](uint32_t (&sr)[128], int i) {
         tmem_ld32(tS + 0, sr);
         tmem_ld32(tS + 32, sr + 32);
         tmem_ld32(tS + 64, sr + 64);
@@ -251,57 +258,83 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           for (int c = 0; c < 128; ++c)
             if (c < vlo || c > vhi) sr[c] = __float_as_uint(-INFINITY);
         }
-        // row max: four independent chains of three-input maxima, then a tree
-        float mx4[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1]));
-#pragma unroll
-        for (int c = 8; c < 128; c += 8)
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            mx4[u] = max3(mx4[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        const float mxs = mx * sl2;
-        const bool need = mxs > m_used + kRescaleThreshold;
-        if (i > 0 && __any_sync(0xffffffffu, need)) {
-          const float f = need ? exp2f(m_used - mxs) : 1.f;
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t o[32];
-            tmem_ld32(tO + cc * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-            tmem_st32(tO + cc * 32, o);
-          }
-          tmem_wait_st();
-        }
-        if (need) {
-          l *= exp2f(m_used - mxs);
-          m_used = mxs;
-        }
-        // a row with no valid key yet keeps m_used = -inf: use 0 as the base (p = 0)
-        const float mb = m_used == -INFINITY ? 0.f : m_used;
-        // x = s * scale * log2(e) - base and the row sum run as packed pairs
+      };
+      // p = 2^(s * scale * log2(e) - mb) as bf16 pairs; returns the fp32 sum of p
+      auto exp_tile = [&](const uint32_t (&sr)[128], float mb, uint32_t (&pk)[64]) -> float {
         const uint64_t sl2x2 = f2_pack(sl2, sl2), nmbx2 = f2_pack(-mb, -mb);
         uint64_t rs4[4] = {0ull, 0ull, 0ull, 0ull};
-        uint32_t pk[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2, nmbx2),
-                    x0, x1);
-          const bool poly = kPolyPeriod > 0 && (c % (kPolyPeriod > 0 ? kPolyPeriod : 1)) == kPolyPeriod - 1;
-          const float p0 = poly ? exp2_poly(x0) : ex2(x0);
-          const float p1 = poly ? exp2_poly(x1) : ex2(x1);
-          rs4[c & 3] = f2_add(rs4[c & 3], f2_pack(p0, p1));
+          const uint64_t x2 =
+              f2_fma(f2_pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2, nmbx2);
+          uint64_t p2;
+          if (((c * kPolyOf8) & 7) < kPolyOf8) {
+            p2 = exp2_poly2(x2);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p2 = f2_pack(ex2(x0), ex2(x1));
+          }
+          rs4[c & 3] = f2_add(rs4[c & 3], p2);
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
           pk[c] = pack_bf16x2(p0, p1);
         }
-        {
-          float a0, a1;
-          f2_unpack(f2_add(f2_add(rs4[0], rs4[1]), f2_add(rs4[2], rs4[3])), a0, a1);
-          l += a0 + a1;
+        float a0, a1;
+        f2_unpack(f2_add(f2_add(rs4[0], rs4[1]), f2_add(rs4[2], rs4[3])), a0, a1);
+        return a0 + a1;
+      };
+      for (int i = 0; i < nkt && ok; ++i) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.s_full[w]), i & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[128], pk[64];
+        float ts = 0.f;
+        load_s(sr, i);
+        // fast path: exponentials against the current base m_used, no row max;
+        // taken back (S reloaded from TMEM) if any row of the warp sums above
+        // the limit or has no base yet
+        bool slow = __any_sync(0xffffffffu, m_used == -INFINITY);
+        if (!slow) {
+          ts = exp_tile(sr, m_used, pk);
+          slow = __any_sync(0xffffffffu, !(ts <= kFastSumLimit));
+          if (slow) load_s(sr, i);
         }
+        if (slow) {
+          // row max: four independent chains of three-input maxima, then a tree
+          float mx4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(__uint_as_float(sr[2 * u]), __uint_as_float(sr[2 * u + 1]));
+#pragma unroll
+          for (int c = 8; c < 128; c += 8)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              mx4[u] = max3(mx4[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
+          const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+          const float mxs = mx * sl2;
+          const bool need = mxs > m_used + kRescaleThreshold;
+          if (i > 0 && __any_sync(0xffffffffu, need)) {
+            // S_i complete implies PV_(i-1) complete (MMA issue order), so O is final here
+            const float f = need ? exp2f(m_used - mxs) : 1.f;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t o[32];
+              tmem_ld32(tO + cc * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+              tmem_st32(tO + cc * 32, o);
+            }
+            tmem_wait_st();
+          }
+          if (need) {
+            l *= exp2f(m_used - mxs);
+            m_used = mxs;
+          }
+          // a row with no valid key yet keeps m_used = -inf: use 0 as the base (p = 0)
+          ts = exp_tile(sr, m_used == -INFINITY ? 0.f : m_used, pk);
+        }
+        l += ts;
         tmem_st32(tS + 0, pk);
         tmem_st32(tS + 32, pk + 32);
         tmem_wait_st();
@@ -341,64 +374,88 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           }
           if (valid) part_lse[pidx] = lse2;
         } else {
-          // merge with the historical partials of the row (Algorithm 1 Step 4)
+          // merge with the historical partials of the row (Algorithm 1 Step 4).
+          // Every MMA has completed, so the Q/K/V buffers are free: each warp
+          // stages the partials of its 32 rows there slot by slot (one cp.async
+          // of the warp copies two rows' 256 contiguous bytes), kMergeStages
+          // slots in flight, and each lane reads its own row back.
           const int nh = valid ? min(KH, t / dm.B) : 0;
           const size_t pbase = (size_t)((b * dm.chunk + (t - t0)) * dm.hq + h) * KH;
+          float pl[MOBA_MAX_TOPK - 1];
           float M = lse2;
-          for (int s = 0; s < nh; ++s) M = fmaxf(M, part_lse[pbase + s]);
+#pragma unroll
+          for (int s = 0; s < MOBA_MAX_TOPK - 1; ++s) {
+            pl[s] = s < nh ? part_lse[pbase + s] : -INFINITY;
+            M = fmaxf(M, pl[s]);
+          }
           const float wc = exp2f(lse2 - M);
           float W = wc;
-          for (int s = 0; s < nh; ++s) W += exp2f(part_lse[pbase + s] - M);
+#pragma unroll
+          for (int s = 0; s < MOBA_MAX_TOPK - 1; ++s) W += exp2f(pl[s] - M);
           const float iw = 1.f / W;
           const float fc = wc / l * iw;
-          __nv_bfloat16* dst = out + (size_t)r * kD;
+          float acc[kD];
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             uint32_t o[32];
             tmem_ld32(tO + cc * 32, o);
             tmem_wait_ld();
-            if (valid) {
-              float acc[32];
 #pragma unroll
-              for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(o[e]) * fc;
-              const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(part_o);
-              // four slots per round so 16 loads are in flight
-              for (int s0 = 0; s0 < nh; s0 += 4) {
-                uint4 x[4][4];
+            for (int e = 0; e < 32; ++e) acc[cc * 32 + e] = __uint_as_float(o[e]) * fc;
+          }
+          fence_proxy_async_smem();
+          const int nhw = __reduce_max_sync(0xffffffffu, nh);
+          const uint32_t stage = base + (uint32_t)warp * kMergeWarpBytes;
+          const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(part_o);
+          // row rr of this warp is token t - lane + rr: its partials start rr * hq * KH slots later
+          const size_t pbase0 = pbase - (size_t)lane * dm.hq * KH;
+          auto issue = [&](int sl) {
+            const uint32_t buf = stage + (uint32_t)(sl % kMergeStages) * kMergeSlotBytes;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  const uint4* src4 =
-                      reinterpret_cast<const uint4*>(pb + (pbase + s0 + u) * kD + cc * 32);
+            for (int k = 0; k < 16; ++k) {
+              const int rr = 2 * k + (lane >> 4), c = lane & 15;
+              const bool live = sl < __shfl_sync(0xffffffffu, nh, rr);
+              const __nv_bfloat16* src = live ? pb + (pbase0 + (size_t)rr * dm.hq * KH + sl) * kD + c * 8 : pb;
+              cp_async16(buf + rr * 256 + ((c ^ (rr & 15)) << 4), src, live);
+            }
+          };
 #pragma unroll
-                  for (int e8 = 0; e8 < 4; ++e8)
-                    x[u][e8] = (s0 + u < nh) ? __ldg(src4 + e8) : make_uint4(0u, 0u, 0u, 0u);
-                }
+          for (int k = 0; k < kMergeStages - 1; ++k) {
+            if (k < nhw) issue(k);
+            cp_async_commit();
+          }
+          for (int sl = 0; sl < nhw; ++sl) {
+            if (sl + kMergeStages - 1 < nhw) issue(sl + kMergeStages - 1);
+            cp_async_commit();
+            cp_async_wait<kMergeStages - 1>();
+            __syncwarp();
+            if (sl < nh) {
+              const float ws = exp2f(part_lse[pbase + sl] - M) * iw;
+              const uint32_t row = stage + (uint32_t)(sl % kMergeStages) * kMergeSlotBytes + lane * 256;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  if (s0 + u < nh) {
-                    const float ws = exp2f(part_lse[pbase + s0 + u] - M) * iw;
+              for (int c = 0; c < 16; ++c) {
+                uint32_t w4[4];
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+                             : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
+                             : "r"(row + ((c ^ (lane & 15)) << 4)));
 #pragma unroll
-                    for (int e8 = 0; e8 < 4; ++e8) {
-                      const uint32_t w4[4] = {x[u][e8].x, x[u][e8].y, x[u][e8].z, x[u][e8].w};
-#pragma unroll
-                      for (int h2 = 0; h2 < 4; ++h2) {
-                        const float2 f2 =
-                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[h2]));
-                        acc[8 * e8 + 2 * h2] = fmaf(ws, f2.x, acc[8 * e8 + 2 * h2]);
-                        acc[8 * e8 + 2 * h2 + 1] = fmaf(ws, f2.y, acc[8 * e8 + 2 * h2 + 1]);
-                      }
-                    }
-                  }
+                for (int h2 = 0; h2 < 4; ++h2) {
+                  const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[h2]));
+                  acc[8 * c + 2 * h2] = fmaf(ws, f2.x, acc[8 * c + 2 * h2]);
+                  acc[8 * c + 2 * h2 + 1] = fmaf(ws, f2.y, acc[8 * c + 2 * h2 + 1]);
                 }
               }
-              uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-              for (int e8 = 0; e8 < 4; ++e8)
-                d4[e8] = make_uint4(pack_bf16x2(acc[8 * e8 + 0], acc[8 * e8 + 1]),
-                                    pack_bf16x2(acc[8 * e8 + 2], acc[8 * e8 + 3]),
-                                    pack_bf16x2(acc[8 * e8 + 4], acc[8 * e8 + 5]),
-                                    pack_bf16x2(acc[8 * e8 + 6], acc[8 * e8 + 7]));
             }
+            __syncwarp();
+          }
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(out + (size_t)r * kD);
+#pragma unroll
+            for (int e8 = 0; e8 < 16; ++e8)
+              d4[e8] = make_uint4(pack_bf16x2(acc[8 * e8 + 0], acc[8 * e8 + 1]),
+                                  pack_bf16x2(acc[8 * e8 + 2], acc[8 * e8 + 3]),
+                                  pack_bf16x2(acc[8 * e8 + 4], acc[8 * e8 + 5]),
+                                  pack_bf16x2(acc[8 * e8 + 6], acc[8 * e8 + 7]));
           }
           if (valid && lse != nullptr)
             lse[((size_t)b * dm.hq + h) * dm.N + t] = (M + log2f(W)) * kLn2;

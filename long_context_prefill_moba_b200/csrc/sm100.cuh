@@ -183,6 +183,11 @@ MOBA_DEV uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+MOBA_DEV uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 MOBA_DEV float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -190,7 +195,7 @@ MOBA_DEV float max3(float a, float b, float c) {
 }
 
 // 2^x on the special-function unit: the PTX approximate base-2 exponential
-// (flush-to-zero; arguments here are <= 8 and results below 2^-126 do not
+// (flush-to-zero; arguments here are <= 15 and results below 2^-126 do not
 // matter for a softmax)
 MOBA_DEV float ex2_approx(float x) {
   float y;
@@ -211,6 +216,28 @@ MOBA_DEV float exp2_poly(float x) {
   const float p = fmaf(fmaf(fmaf(0.05517206f, f, 0.24261241f), f, 0.69326101f), f, 0.99992796f);
   const int n = __float_as_int(r) - 0x4B400000;   // bits of 12582912.f
   return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+// exp2_poly on a packed pair: the same clamp, range reduction, polynomial and
+// exponent insertion, bit for bit, with the fp32 steps as paired instructions
+// (three adds/subtracts and three FMAs per pair on the FMA pipe).
+MOBA_DEV uint64_t exp2_poly2(uint64_t x2) {
+  float a, b;
+  f2_unpack(x2, a, b);
+  const uint64_t xc = f2_pack(fmaxf(a, -126.f), fmaxf(b, -126.f));
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t r = f2_add(xc, magic);
+  const uint64_t f = f2_sub(xc, f2_sub(r, magic));
+  uint64_t p = f2_fma(f2_pack(0.05517206f, 0.05517206f), f, f2_pack(0.24261241f, 0.24261241f));
+  p = f2_fma(p, f, f2_pack(0.69326101f, 0.69326101f));
+  p = f2_fma(p, f, f2_pack(0.99992796f, 0.99992796f));
+  float p0, p1, r0, r1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(r, r0, r1);
+  // (rint(x) << 23) == (bits(r) << 23) modulo 2^32: the low 9 bits of
+  // bits(1.5 * 2^23) are zero
+  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(r0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(r1) << 23)));
 }
 
 // byte offset of the 16-byte chunk `c` (0..7) of row `r` inside a 128-byte
