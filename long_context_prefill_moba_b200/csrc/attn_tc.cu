@@ -498,21 +498,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, kBK, false);
       const uint32_t idO = idesc_bf16(128, kD, true);
+      // descriptor words precomputed once; each MMA adds a compile-time offset
+      const uint32_t hi = sdesc_hi(1024);
+      const uint32_t loQ = sdesc_lo(base + kOffQ, 16), loK = sdesc_lo(base + kOffK, 16),
+                     loV = sdesc_lo(base + kOffV, kHalf);
       auto issue_s = [&](int w, int s) {
-        const uint32_t qa = base + kOffQ + w * kTile, ka = base + kOffK + s * kTile;
+        const uint32_t qa = loQ + (w ? (kTile >> 4) : 0u), ka = loK + (s ? (kTile >> 4) : 0u);
         const uint32_t d = tb + (w ? 128u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          mma_ss(d, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS, kk > 0);
+          const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+          mma_ss(d, sdesc_join(qa + off, hi), sdesc_join(ka + off, hi), idS, kk > 0);
         }
       };
       auto issue_pv = [&](int w, int s, bool acc) {
-        const uint32_t va = base + kOffV + s * kTile;
+        const uint32_t va = loV + (s ? (kTile >> 4) : 0u);
         const uint32_t d = tb + (w ? 384u : 256u), a = tb + (w ? 128u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(d, a + kk * 8, sdesc_sw128(va + kk * 2048, kHalf, 1024), idO, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(d, a + kk * 8, sdesc_join(va + ((kk * 2048) >> 4), hi), idO, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(&ctl.q_full[0]), 0, abort_flag);
       if (ok && nq == 2) ok = mbar_wait(bar(&ctl.q_full[1]), 0, abort_flag);

@@ -125,9 +125,27 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
 // Shared-memory matrix descriptor, 128-byte swizzle:
 // bits [0,14) start >> 4, [16,30) leading-dim byte offset >> 4,
 // [32,46) stride-dim byte offset >> 4, [46,48) version = 1, [61,64) layout 2 (SW128).
-MOBA_DEV uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+__host__ __device__ constexpr uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// The same descriptor as two 32-bit words, so an issue loop can precompute the
+// low word of a tile once and add compile-time offsets (offset >> 4) to it:
+// shared addresses of a CTA stay below 256 KB, so the 14-bit start field
+// never carries into the leading-offset field.
+__host__ __device__ constexpr uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sdesc_hi(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+static_assert(sdesc_sw128(0x2F3C0u + 0x4020u, 16384, 1024) ==
+                  (((uint64_t)sdesc_hi(1024) << 32) | (sdesc_lo(0x2F3C0u, 16384) + (0x4020u >> 4))),
+              "split descriptor words");
+MOBA_DEV uint64_t sdesc_join(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
 }
 
 // ---- tcgen05: TMEM <-> registers (32 lanes x 32-bit, 32 columns per thread) --
