@@ -182,6 +182,39 @@ MOBA_API moba_status_t moba_attn_fwd(const moba_shape_t* shape, const void* q, c
                                      const int32_t* rows, void* out, float* lse, void* ws,
                                      size_t ws_bytes, moba_stream_t stream);
 
+/* ---- the whole layer from host buffers ---------------------------------- */
+
+/* Device bytes moba_prefill_host needs for `shape` (with_lse: whether an lse
+ * output will be requested); 0 for an invalid shape. */
+MOBA_API size_t moba_prefill_host_workspace_size(const moba_shape_t* shape, int with_lse);
+
+/* One MoBA prefill layer (Algorithm 1, Steps 1-4: mean-pool, gate, block-sparse
+ * attention, merge; the same kernels and results as moba_block_meanpool +
+ * moba_gate_topk + moba_attn_fwd) from and to HOST buffers, with the copies
+ * overlapped with the computation.  The paper has no counterpart: this is the
+ * library's host-side runtime around the three steps.
+ *   q, k, v  host [batch, seqlen, hq|hkv, head_dim] dtype   (read)
+ *   out      host [batch, seqlen, hq, head_dim] dtype       (written)
+ *   lse      host [batch, hq, seqlen] fp32 natural log, or NULL (written)
+ *   status   host int[2], or NULL: after the stream completes, the gate's and
+ *            the attention's device status words (0, or MOBA_ERR_TIMEOUT)
+ *   ws       >= moba_prefill_host_workspace_size(shape, lse != NULL) bytes of
+ *            device memory, 16-byte aligned; it holds the device copies of the
+ *            tensors and every intermediate array
+ * k and v are copied in first (mean-pool starts when they land); q arrives one
+ * query pass (moba_query_chunk tokens) at a time on a second stream, the gate
+ * and the attention of a pass start as soon as its queries are in, and each
+ * pass's output returns on a third stream while the next pass computes.  The
+ * call only enqueues: `stream` (the compute stream) completes when the last
+ * output byte is in host memory.  The copies overlap only from page-locked
+ * host memory (cudaHostAlloc / cudaHostRegister); pageable buffers give the
+ * same results with copies that block the calling thread.  The call creates
+ * and releases two streams and 2 * (passes + 2) events; it does no device
+ * allocation. */
+MOBA_API moba_status_t moba_prefill_host(const moba_shape_t* shape, const void* q, const void* k,
+                                         const void* v, void* out, float* lse, int* status,
+                                         void* ws, size_t ws_bytes, moba_stream_t stream);
+
 /* ---- diagnostics ------------------------------------------------------- */
 
 /* Static description of a status code. */

@@ -31,6 +31,7 @@ __all__ = [
     "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems", "moba_gate_workspace_size",
     "moba_attn_workspace_size", "moba_block_meanpool", "moba_gate_topk", "moba_attn_fwd",
     "moba_status_string", "moba_last_launch_count", "moba_gate_topk_noalloc", "MobaLayer", "moba_forward",
+    "moba_prefill_host_workspace_size", "moba_prefill_host", "MobaHostLayer",
     "MOBA_BF16", "MOBA_F32", "EXPORTED_SYMBOLS",
 ]
 
@@ -46,6 +47,7 @@ EXPORTED_SYMBOLS = [
     "moba_gate_workspace_size", "moba_attn_workspace_size", "moba_block_meanpool",
     "moba_gate_topk", "moba_attn_fwd", "moba_status_string", "moba_last_cuda_error",
     "moba_last_launch_count", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait",
+    "moba_prefill_host_workspace_size", "moba_prefill_host",
 ]
 
 
@@ -103,6 +105,10 @@ def load_library(path: str = LIB_PATH):
     L.moba_selftest_bounded_wait.restype = st
     L.moba_gate_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
     L.moba_gate_topk_noalloc.restype = st
+    L.moba_prefill_host_workspace_size.argtypes = [P, st]
+    L.moba_prefill_host_workspace_size.restype = sz
+    L.moba_prefill_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moba_prefill_host.restype = st
     L.moba_status_string.argtypes = [st]
     L.moba_status_string.restype = ctypes.c_char_p
     L.moba_last_cuda_error.argtypes = []
@@ -191,6 +197,60 @@ def moba_attn_fwd(shape, q, k, v, sel, offsets, rows, out, lse, ws, stream=None)
                                _ptr(rows), _ptr(out), _ptr(lse), _ptr(ws),
                                ws.numel() * ws.element_size(), _stream(stream)),
            "moba_attn_fwd")
+
+
+def moba_prefill_host_workspace_size(shape, with_lse=False) -> int:
+    return lib().moba_prefill_host_workspace_size(_s(shape), 1 if with_lse else 0)
+
+
+def moba_prefill_host(shape, q, k, v, out, lse, status, ws, stream=None):
+    """One layer from host tensors (q, k, v, out, lse: CPU, contiguous; page-locked
+    for the copies to overlap the computation); `status` a 2-element CPU int32
+    tensor or None; `ws` a CUDA byte tensor of moba_prefill_host_workspace_size."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("status", status)):
+        if t is not None and t.device.type != "cpu":
+            raise ValueError(f"moba_prefill_host: {name} must be a host tensor")
+    if ws.device.type != "cuda":
+        raise ValueError("moba_prefill_host: ws must be device memory")
+    _check(lib().moba_prefill_host(_s(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                   _ptr(status), _ptr(ws), ws.numel() * ws.element_size(),
+                                   _stream(stream)),
+           "moba_prefill_host")
+
+
+class MobaHostLayer:
+    """One MoBA layer shape served from host buffers (moba_prefill_host): the
+    device workspace is allocated once; ``forward`` enqueues the copies and the
+    three steps with the copies overlapped, on the current stream."""
+
+    def __init__(self, batch, seqlen, hq, hkv, head_dim, block, topk, dtype="bf16", scale=None,
+                 query_chunk=0, device="cuda", with_lse=False):
+        self.shape = make_shape(batch, seqlen, hq, hkv, head_dim, block, topk, dtype, scale,
+                                query_chunk)
+        _check(moba_check_shape(self.shape), "MobaHostLayer")
+        self.device = torch.device(device)
+        self.with_lse = with_lse
+        self.ws = torch.empty(moba_prefill_host_workspace_size(self.shape, with_lse), dtype=torch.uint8,
+                              device=self.device)
+        self.status = torch.zeros(2, dtype=torch.int32, pin_memory=True)
+        self.launches = 0
+
+    @classmethod
+    def from_config(cls, cfg, device="cuda", query_chunk=0, with_lse=False):
+        return cls(cfg.batch, cfg.seqlen, cfg.hq, cfg.hkv, cfg.head_dim, cfg.block, cfg.topk,
+                   cfg.dtype, cfg.scale, query_chunk, device, with_lse)
+
+    def forward(self, q, k, v, out, lse=None, stream=None):
+        if lse is not None and not self.with_lse:
+            raise ValueError("MobaHostLayer: built without an lse output")
+        moba_prefill_host(self.shape, q, k, v, out, lse, self.status, self.ws, stream)
+        self.launches = moba_last_launch_count()
+        return out
+
+    def device_status(self):
+        """(gate, attention) status words of the last forward (synchronises)."""
+        torch.cuda.synchronize(self.device)
+        return int(self.status[0]), int(self.status[1])
 
 
 class MobaLayer:

@@ -39,17 +39,17 @@ int64_t hist_rows_range(int64_t t0, int64_t t1, int64_t B, int64_t KH) {
   return total;
 }
 
-cudaError_t launch_attn(const Dims& dm, int dtype, const void* q, const void* k, const void* v,
-                        const int32_t* sel, const int32_t* offsets, const int32_t* rows, void* out,
-                        float* lse, AttnWs ws, cudaStream_t stream, int* launches) {
+cudaError_t launch_attn_passes(const Dims& dm, int dtype, const void* q, const void* k,
+                               const void* v, const int32_t* sel, const int32_t* offsets,
+                               const int32_t* rows, void* out, float* lse, AttnWs ws, int ch_begin,
+                               int ch_end, cudaStream_t stream, int* launches) {
   const int KH = dm.topk - 1;
   const int ngroups = dm.batch * dm.hkv * dm.n;
-  cudaError_t e = cudaMemsetAsync(ws.status, 0, sizeof(int), stream);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   // bf16 with head_dim 128: tensor-core (tcgen05) kernels for both attention steps
   const bool tc = dtype == MOBA_BF16 && dm.d == 128;
   const int tm = tc ? attn_tc_rows_per_tile() : 64;
-  for (int ch = 0; ch < dm.nchunks; ++ch) {
+  for (int ch = ch_begin; ch < ch_end; ++ch) {
     const int t0 = ch * dm.chunk;
     const int t1 = dm.N < t0 + dm.chunk ? dm.N : t0 + dm.chunk;
     const int64_t nrows = hist_rows_range(t0, t1, dm.B, KH) * dm.batch * dm.hq;
@@ -77,6 +77,15 @@ cudaError_t launch_attn(const Dims& dm, int dtype, const void* q, const void* k,
     if (e != cudaSuccess) return e;
   }
   return e;
+}
+
+cudaError_t launch_attn(const Dims& dm, int dtype, const void* q, const void* k, const void* v,
+                        const int32_t* sel, const int32_t* offsets, const int32_t* rows, void* out,
+                        float* lse, AttnWs ws, cudaStream_t stream, int* launches) {
+  cudaError_t e = cudaMemsetAsync(ws.status, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return e;
+  return launch_attn_passes(dm, dtype, q, k, v, sel, offsets, rows, out, lse, ws, 0, dm.nchunks,
+                            stream, launches);
 }
 
 }  // namespace moba

@@ -19,6 +19,7 @@ struct Dims {
   int batch, N, hq, hkv, d, B, topk, n, G;
   int chunk;        // tokens per attention pass
   int nchunks;
+  int t_lo, t_hi;   // token window [t_lo, t_hi) of the gate kernels (t_lo a multiple of 128)
   float scale_log2; // softmax scale * log2(e)
 };
 

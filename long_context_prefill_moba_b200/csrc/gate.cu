@@ -36,17 +36,17 @@ __global__ void __launch_bounds__(kRows) gate_select_kernel(const T* __restrict_
                                                             int32_t* __restrict__ counts, Dims dm) {
   __shared__ __align__(16) float kb[kJChunk * D];
   __shared__ int hist[kSmemHist];
-  const int tiles_per_seq = (dm.N + kRows - 1) / kRows;
+  const int tiles_per_seq = (dm.t_hi - dm.t_lo + kRows - 1) / kRows;
   const int tile = blockIdx.x % tiles_per_seq;
   const int bh = blockIdx.x / tiles_per_seq;
   const int h = bh % dm.hq;
   const int b = bh / dm.hq;
   const int g = h / dm.G;
-  const int t_first = tile * kRows;
+  const int t_first = dm.t_lo + tile * kRows;
   const int t = t_first + threadIdx.x;
-  const bool valid = t < dm.N;
+  const bool valid = t < dm.t_hi;
   const int c = valid ? t / dm.B : 0;
-  const int t_last = min(dm.N, t_first + kRows) - 1;
+  const int t_last = min(dm.t_hi, t_first + kRows) - 1;
   const int c_max = t_last / dm.B;              // largest current block in the tile
   const int KH = dm.topk - 1;                   // historical slots
   const bool use_hist = dm.n <= kSmemHist;
@@ -155,14 +155,14 @@ __global__ void __launch_bounds__(kRows) gate_select_kernel(const T* __restrict_
   }
 }
 
-// Exclusive prefix sum of `in` (len L) into out[0..L]; one CTA.
+// Exclusive prefix sum of `in` (len L) plus `base` into out[0..L]; one CTA.
 constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads) gate_scan_kernel(const int32_t* __restrict__ in,
                                                                  int32_t* __restrict__ out,
-                                                                 int64_t L) {
+                                                                 int64_t L, int32_t base) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t carry;
-  if (threadIdx.x == 0) carry = 0;
+  if (threadIdx.x == 0) carry = base;
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int64_t base = 0; base < L; base += kScanThreads) {
@@ -201,16 +201,16 @@ __global__ void __launch_bounds__(kRows) gate_scatter_kernel(const int32_t* __re
                                                              int32_t* __restrict__ rows, Dims dm) {
   __shared__ int cnt[kSmemHist];
   __shared__ int base[kSmemHist];
-  const int tiles_per_seq = (dm.N + kRows - 1) / kRows;
+  const int tiles_per_seq = (dm.t_hi - dm.t_lo + kRows - 1) / kRows;
   const int tile = blockIdx.x % tiles_per_seq;
   const int bh = blockIdx.x / tiles_per_seq;
   const int h = bh % dm.hq;
   const int b = bh / dm.hq;
   const int g = h / dm.G;
-  const int t_first = tile * kRows;
+  const int t_first = dm.t_lo + tile * kRows;
   const int t = t_first + threadIdx.x;
-  const bool valid = t < dm.N;
-  const int t_last = min(dm.N, t_first + kRows) - 1;
+  const bool valid = t < dm.t_hi;
+  const int t_last = min(dm.t_hi, t_first + kRows) - 1;
   const int c_max = t_last / dm.B;
   const int KH = dm.topk - 1;
   const bool use_hist = dm.n <= kSmemHist;
@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kRows) gate_scatter_kernel(const int32_t* __re
 template <typename T>
 cudaError_t launch_select(const Dims& dm, const void* q, const float* meank, int32_t* sel,
                           int32_t* counts, cudaStream_t stream) {
-  const int tiles = (dm.N + kRows - 1) / kRows;
+  const int tiles = (dm.t_hi - dm.t_lo + kRows - 1) / kRows;
   dim3 grid(tiles * dm.batch * dm.hq);
   if (dm.d == 128)
     gate_select_kernel<T, 128><<<grid, kRows, 0, stream>>>(static_cast<const T*>(q), meank, sel,
@@ -278,11 +278,43 @@ cudaError_t launch_gate(const Dims& dm, int dtype, const void* q, const float* m
     e = launch_select<float>(dm, q, meank, sel, ws.counts, stream);
   ++*launches;
   if (e != cudaSuccess) return e;
-  gate_scan_kernel<<<1, kScanThreads, 0, stream>>>(ws.counts, offsets, L);
+  gate_scan_kernel<<<1, kScanThreads, 0, stream>>>(ws.counts, offsets, L, 0);
   ++*launches;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (dm.topk > 1) {
-    const int tiles = (dm.N + kRows - 1) / kRows;
+    const int tiles = (dm.t_hi - dm.t_lo + kRows - 1) / kRows;
+    gate_scatter_kernel<<<tiles * dm.batch * dm.hq, kRows, 0, stream>>>(sel, offsets, ws.cursors,
+                                                                        rows, dm);
+    ++*launches;
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+cudaError_t launch_gate_pass(const Dims& dm_all, int dtype, const void* q, const float* meank,
+                             int32_t* sel, int32_t* offsets, int32_t* rows, GateWs ws, int pass,
+                             cudaStream_t stream, int* launches) {
+  Dims dm = dm_all;
+  dm.t_lo = pass * dm.chunk;
+  dm.t_hi = dm.N < dm.t_lo + dm.chunk ? dm.N : dm.t_lo + dm.chunk;
+  const int64_t G0 = (int64_t)dm.batch * dm.hkv * dm.n;   // groups of one pass
+  // rows of the earlier passes: every token t contributes min(topk - 1, t / B) per (b, h)
+  const int64_t before = hist_rows_range(0, dm.t_lo, dm.B, dm.topk - 1) * dm.batch * dm.hq;
+  cudaError_t e;
+  if (gate_tc_supported(dm, dtype))
+    e = launch_gate_select_tc(dm, q, meank, sel, ws.counts, ws.status, stream);
+  else if (dtype == MOBA_BF16)
+    e = launch_select<__nv_bfloat16>(dm, q, meank, sel, ws.counts, stream);
+  else
+    e = launch_select<float>(dm, q, meank, sel, ws.counts, stream);
+  ++*launches;
+  if (e != cudaSuccess) return e;
+  gate_scan_kernel<<<1, kScanThreads, 0, stream>>>(ws.counts + pass * G0, offsets + pass * G0, G0,
+                                                   (int32_t)before);
+  ++*launches;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (dm.topk > 1) {
+    const int tiles = (dm.t_hi - dm.t_lo + kRows - 1) / kRows;
     gate_scatter_kernel<<<tiles * dm.batch * dm.hq, kRows, 0, stream>>>(sel, offsets, ws.cursors,
                                                                         rows, dm);
     ++*launches;

@@ -77,12 +77,12 @@ __global__ void __launch_bounds__(kThreads, 1) gate_select_tc_kernel(
   extern __shared__ uint8_t smem_raw[];
   __shared__ Ctl ctl;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const int ranges = (dm.N + kTokens - 1) / kTokens;
+  const int ranges = (dm.t_hi - dm.t_lo + kTokens - 1) / kTokens;
   const int rg = blockIdx.x % ranges;
   const int g = (blockIdx.x / ranges) % dm.hkv;
   const int b = blockIdx.x / (ranges * dm.hkv);
-  const int t_begin = rg * kTokens;
-  const int t_stop = min(dm.N, t_begin + kTokens);
+  const int t_begin = dm.t_lo + rg * kTokens;
+  const int t_stop = min(dm.t_hi, t_begin + kTokens);
   const int ttiles = (t_stop - t_begin + kRowsT - 1) / kRowsT;
   const int ntiles = ttiles * dm.G;                 // tile k: token tile k / G, head g*G + k % G
   const int cmax_cta = (t_stop - 1) / dm.B;         // blocks [0, cmax_cta) may be candidates
@@ -150,9 +150,9 @@ __global__ void __launch_bounds__(kThreads, 1) gate_select_tc_kernel(
       const int tt = t_begin + (k / dm.G) * kRowsT;
       const int h = g * dm.G + k % dm.G;
       const int t = tt + rho;
-      const bool valid = t < dm.N;
+      const bool valid = t < dm.t_hi;
       const int c = valid ? t / dm.B : 0;
-      const int ctile = (min(dm.N, tt + kRowsT) - 1) / dm.B;   // candidates of the tile: [0, ctile)
+      const int ctile = (min(dm.t_hi, tt + kRowsT) - 1) / dm.B;   // candidates of the tile: [0, ctile)
       // the decision is uniform over the four selection warps, so the named
       // barriers below are always reached by all of them
       ok = selectors_all(mbar_wait(bar(&ctl.s_full[k & 1]), (k >> 1) & 1, abort_flag));
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_select_tc_kernel(
       for (int k = 0; k < ntiles && ok; ++k) {
         const int s = k & 1;
         const int tt = t_begin + (k / dm.G) * kRowsT;
-        const int ctile = (min(dm.N, tt + kRowsT) - 1) / dm.B;
+        const int ctile = (min(dm.t_hi, tt + kRowsT) - 1) / dm.B;
         const int nt = max(16, (ctile + 15) / 16 * 16);
         ok = mbar_wait(bar(&ctl.q_full[s]), (k >> 1) & 1, abort_flag);
         if (ok && k >= 2) ok = mbar_wait(bar(&ctl.s_free[s]), ((k >> 1) - 1) & 1, abort_flag);
@@ -303,7 +303,7 @@ cudaError_t run_select(const CUtensorMap& mq, const Dims& dm, const float* meank
   cudaError_t e = cudaFuncSetAttribute(gate_select_tc_kernel<KB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int ranges = (dm.N + kTokens - 1) / kTokens;
+  const int ranges = (dm.t_hi - dm.t_lo + kTokens - 1) / kTokens;
   gate_select_tc_kernel<KB><<<(int64_t)ranges * dm.hkv * dm.batch, kThreads, kSmemBytes, stream>>>(
       mq, meank, sel, counts, status, dm);
   return cudaGetLastError();

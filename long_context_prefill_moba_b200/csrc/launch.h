@@ -32,6 +32,13 @@ cudaError_t launch_gate(const Dims& dm, int dtype, const void* q, const float* m
                         int32_t* offsets, int32_t* rows, GateWs ws, cudaStream_t stream,
                         int* launches);
 
+// the gate of one query pass (tokens [pass * chunk, +chunk)): selection,
+// offsets of that pass's groups (continuing the earlier passes' rows) and the
+// scatter; the counters of ws must be zero beforehand
+cudaError_t launch_gate_pass(const Dims& dm, int dtype, const void* q, const float* meank,
+                             int32_t* sel, int32_t* offsets, int32_t* rows, GateWs ws, int pass,
+                             cudaStream_t stream, int* launches);
+
 // moba_gate_topk with the counters in the library's fixed device array
 // (requires nchunks * batch * hkv * n <= MOBA_GATE_NOALLOC_MAX_GROUPS)
 cudaError_t launch_gate_noalloc(const Dims& dm, int dtype, const void* q, const float* meank,
@@ -47,6 +54,11 @@ struct AttnWs {
 cudaError_t launch_attn(const Dims& dm, int dtype, const void* q, const void* k, const void* v,
                         const int32_t* sel, const int32_t* offsets, const int32_t* rows, void* out,
                         float* lse, AttnWs ws, cudaStream_t stream, int* launches);
+// passes [ch_begin, ch_end) only, without resetting the status word
+cudaError_t launch_attn_passes(const Dims& dm, int dtype, const void* q, const void* k,
+                               const void* v, const int32_t* sel, const int32_t* offsets,
+                               const int32_t* rows, void* out, float* lse, AttnWs ws, int ch_begin,
+                               int ch_end, cudaStream_t stream, int* launches);
 
 // a kernel whose only wait can never complete: it must time out (status word)
 cudaError_t launch_bounded_wait_selftest(int* status, cudaStream_t stream);

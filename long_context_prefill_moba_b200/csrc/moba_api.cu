@@ -56,6 +56,8 @@ moba::Dims make_dims(const moba_shape_t* s) {
   d.G = s->hq / s->hkv;
   d.chunk = (int)chunk_of(s);
   d.nchunks = (int)nchunks_of(s);
+  d.t_lo = 0;
+  d.t_hi = s->seqlen;
   const float scale = s->scale > 0.f ? s->scale : 1.0f / sqrtf((float)s->head_dim);
   d.scale_log2 = scale * moba::kLog2e;
   return d;
@@ -75,6 +77,33 @@ AttnLayout attn_layout(const moba_shape_t* s) {
   L.part_lse = L.part_o + align_up(entries * s->head_dim * sizeof(float));
   L.tile_start = L.part_lse + align_up(entries * sizeof(float));
   L.total = L.tile_start + align_up(((size_t)s->batch * s->hkv * nblocks(s) + 1) * sizeof(int32_t));
+  return L;
+}
+
+// device workspace of moba_prefill_host: the device copies of q, k, v, out
+// (and lse), then the intermediate arrays and the two step workspaces
+struct HostLayout {
+  size_t q, k, v, out, lse, meank, sel, offsets, rows, gate_ws, attn_ws, total;
+};
+HostLayout host_layout(const moba_shape_t* s, bool with_lse) {
+  const size_t es = s->dtype == MOBA_BF16 ? 2 : 4;
+  const size_t qbytes = (size_t)s->batch * s->seqlen * s->hq * s->head_dim * es;
+  const size_t kbytes = (size_t)s->batch * s->seqlen * s->hkv * s->head_dim * es;
+  HostLayout L;
+  size_t at = 0;
+  auto take = [&](size_t bytes) { const size_t here = at; at += align_up(bytes > 0 ? bytes : 1); return here; };
+  L.q = take(qbytes);
+  L.k = take(kbytes);
+  L.v = take(kbytes);
+  L.out = take(qbytes);
+  L.lse = take(with_lse ? (size_t)s->batch * s->hq * s->seqlen * sizeof(float) : 0);
+  L.meank = take((size_t)s->batch * nblocks(s) * s->hkv * s->head_dim * sizeof(float));
+  L.sel = take((size_t)s->batch * s->seqlen * s->hq * s->topk * sizeof(int32_t));
+  L.offsets = take(((size_t)ngroups_total(s) + 1) * sizeof(int32_t));
+  L.rows = take((size_t)rows_total(s) * sizeof(int32_t));
+  L.gate_ws = take(align_up(2 * (size_t)ngroups_total(s) * sizeof(int32_t)) + 256);
+  L.attn_ws = take(attn_layout(s).total);
+  L.total = at;
   return L;
 }
 
@@ -218,6 +247,129 @@ MOBA_API moba_status_t moba_gate_topk_noalloc(const moba_shape_t* s, const void*
   int launches = 0;
   cudaError_t e = moba::launch_gate_noalloc(make_dims(s), s->dtype, q, meank, sel, offsets, rows,
                                             (cudaStream_t)stream, &launches);
+  return finish(e, launches);
+}
+
+MOBA_API size_t moba_prefill_host_workspace_size(const moba_shape_t* s, int with_lse) {
+  if (moba_check_shape(s) != MOBA_OK) return 0;
+  return host_layout(s, with_lse != 0).total;
+}
+
+MOBA_API moba_status_t moba_prefill_host(const moba_shape_t* s, const void* q, const void* k,
+                                         const void* v, void* out, float* lse, int* status,
+                                         void* ws, size_t ws_bytes, moba_stream_t stream_) {
+  g_last_launches = 0;
+  moba_status_t st = moba_check_shape(s);
+  if (st != MOBA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || ws == nullptr)
+    return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return MOBA_ERR_INVALID_ARG;
+  const HostLayout L = host_layout(s, lse != nullptr);
+  if (ws_bytes < L.total) return MOBA_ERR_WORKSPACE;
+  const moba::Dims dm = make_dims(s);
+  const cudaStream_t stream = (cudaStream_t)stream_;
+  char* base = static_cast<char*>(ws);
+  void* qd = base + L.q;
+  void* kd = base + L.k;
+  void* vd = base + L.v;
+  void* od = base + L.out;
+  float* lsed = lse != nullptr ? reinterpret_cast<float*>(base + L.lse) : nullptr;
+  float* meank = reinterpret_cast<float*>(base + L.meank);
+  int32_t* sel = reinterpret_cast<int32_t*>(base + L.sel);
+  int32_t* offsets = reinterpret_cast<int32_t*>(base + L.offsets);
+  int32_t* rows = reinterpret_cast<int32_t*>(base + L.rows);
+  const int64_t G = ngroups_total(s);
+  moba::GateWs g{reinterpret_cast<int32_t*>(base + L.gate_ws),
+                 reinterpret_cast<int32_t*>(base + L.gate_ws) + G,
+                 reinterpret_cast<int*>(base + L.gate_ws + align_up(2 * (size_t)G * sizeof(int32_t)))};
+  const AttnLayout AL = attn_layout(s);
+  char* ab = base + L.attn_ws;
+  moba::AttnWs a{reinterpret_cast<int*>(ab + AL.status), reinterpret_cast<float*>(ab + AL.part_o),
+                 reinterpret_cast<float*>(ab + AL.part_lse), reinterpret_cast<int32_t*>(ab + AL.tile_start)};
+
+  const size_t es = s->dtype == MOBA_BF16 ? 2 : 4;
+  const size_t qrow = (size_t)s->hq * s->head_dim * es;       // bytes of one token of q / out
+  const size_t kbytes = (size_t)s->batch * s->seqlen * s->hkv * s->head_dim * es;
+  const int np = dm.nchunks;
+
+  // copy-in and copy-out streams beside the caller's compute stream; every
+  // object made here is released at the end (destroying a stream or event
+  // with work pending is legal: it goes once that work is done)
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_kv = nullptr, ev_done = nullptr;
+  cudaEvent_t* ev_q = new cudaEvent_t[np]();
+  cudaEvent_t* ev_o = new cudaEvent_t[np]();
+  int launches = 0;
+  cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+  for (cudaEvent_t* ev : {&ev_start, &ev_kv, &ev_done})
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  for (int p = 0; p < np && e == cudaSuccess; ++p) {
+    e = cudaEventCreateWithFlags(&ev_q[p], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_o[p], cudaEventDisableTiming);
+  }
+  // the copies start after the work already queued on the caller's stream
+  if (e == cudaSuccess) e = cudaEventRecord(ev_start, stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_start, 0);
+  // host -> device: k and v whole, then q one query pass at a time
+  if (e == cudaSuccess) e = cudaMemcpyAsync(kd, k, kbytes, cudaMemcpyHostToDevice, s_in);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(vd, v, kbytes, cudaMemcpyHostToDevice, s_in);
+  if (e == cudaSuccess) e = cudaEventRecord(ev_kv, s_in);
+  for (int p = 0; p < np && e == cudaSuccess; ++p) {
+    const int t0 = p * dm.chunk, t1 = dm.N < t0 + dm.chunk ? dm.N : t0 + dm.chunk;
+    const size_t pitch = (size_t)dm.N * qrow;
+    e = cudaMemcpy2DAsync(static_cast<char*>(qd) + (size_t)t0 * qrow, pitch,
+                          static_cast<const char*>(q) + (size_t)t0 * qrow, pitch, (size_t)(t1 - t0) * qrow,
+                          dm.batch, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_q[p], s_in);
+  }
+  // compute on the caller's stream: mean-pool once k is in, then gate and
+  // attention pass by pass as each pass's queries arrive
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, ev_kv, 0);
+  if (e == cudaSuccess) e = moba::launch_meanpool(dm, s->dtype, kd, meank, stream, &launches);
+  if (e == cudaSuccess) e = cudaMemsetAsync(g.counts, 0, sizeof(int32_t) * G * 2, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(g.status, 0, sizeof(int), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(a.status, 0, sizeof(int), stream);
+  for (int p = 0; p < np && e == cudaSuccess; ++p) {
+    const int t0 = p * dm.chunk, t1 = dm.N < t0 + dm.chunk ? dm.N : t0 + dm.chunk;
+    e = cudaStreamWaitEvent(stream, ev_q[p], 0);
+    if (e == cudaSuccess)
+      e = moba::launch_gate_pass(dm, s->dtype, qd, meank, sel, offsets, rows, g, p, stream, &launches);
+    if (e == cudaSuccess)
+      e = moba::launch_attn_passes(dm, s->dtype, qd, kd, vd, sel, offsets, rows, od, lsed, a, p, p + 1,
+                                   stream, &launches);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_o[p], stream);
+    // device -> host: this pass's output while the next pass computes
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_o[p], 0);
+    if (e == cudaSuccess) {
+      const size_t pitch = (size_t)dm.N * qrow;
+      e = cudaMemcpy2DAsync(static_cast<char*>(out) + (size_t)t0 * qrow, pitch,
+                            static_cast<const char*>(od) + (size_t)t0 * qrow, pitch,
+                            (size_t)(t1 - t0) * qrow, dm.batch, cudaMemcpyDeviceToHost, s_out);
+    }
+    if (e == cudaSuccess && lse != nullptr)
+      e = cudaMemcpy2DAsync(lse + t0, (size_t)dm.N * sizeof(float), lsed + t0, (size_t)dm.N * sizeof(float),
+                            (size_t)(t1 - t0) * sizeof(float), (size_t)dm.batch * dm.hq,
+                            cudaMemcpyDeviceToHost, s_out);
+  }
+  if (e == cudaSuccess && status != nullptr) {
+    e = cudaMemcpyAsync(status, g.status, sizeof(int), cudaMemcpyDeviceToHost, s_out);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(status + 1, a.status, sizeof(int), cudaMemcpyDeviceToHost, s_out);
+  }
+  // the caller's stream completes only after the last copy-out
+  if (e == cudaSuccess) e = cudaEventRecord(ev_done, s_out);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, ev_done, 0);
+  for (int p = 0; p < np; ++p) {
+    if (ev_q[p] != nullptr) cudaEventDestroy(ev_q[p]);
+    if (ev_o[p] != nullptr) cudaEventDestroy(ev_o[p]);
+  }
+  delete[] ev_q;
+  delete[] ev_o;
+  for (cudaEvent_t ev : {ev_start, ev_kv, ev_done})
+    if (ev != nullptr) cudaEventDestroy(ev);
+  if (s_in != nullptr) cudaStreamDestroy(s_in);
+  if (s_out != nullptr) cudaStreamDestroy(s_out);
   return finish(e, launches);
 }
 
