@@ -182,6 +182,36 @@ MOBA_API moba_status_t moba_attn_fwd(const moba_shape_t* shape, const void* q, c
                                      const int32_t* rows, void* out, float* lse, void* ws,
                                      size_t ws_bytes, moba_stream_t stream);
 
+/* ---- backward ---------------------------------------------------------- */
+
+/* Device scratch bytes moba_attn_bwd needs for `shape`; 0 for an invalid shape. */
+MOBA_API size_t moba_attn_bwd_workspace_size(const moba_shape_t* shape);
+
+/* Gradients of the attention step ([summary] §3 "The Core MoBA Attention
+ * Equation" differentiated with the gate's selection held fixed: a top-k of
+ * scores is piecewise constant, so no gradient flows through the routing; the
+ * pages print no backward formula).  For a row r with logits
+ * z_u = scale <q_r, k_u> over its key set and the forward's lse L_r:
+ *   p = exp(z - L_r), D_r = <dout_r, out_r>, ds = p (<dout_r, v_u> - D_r),
+ *   dq_r = scale sum_u ds k_u, dk_u = scale sum_r ds q_r, dv_u = sum_r p dout_r
+ * (query heads of a GQA group add into their kv head's dk, dv).
+ *   q, k, v, sel, offsets, rows  as for moba_attn_fwd                (read)
+ *   out   [batch, seqlen, hq, head_dim] dtype: the forward's output  (read)
+ *   dout  [batch, seqlen, hq, head_dim] dtype: dL/d(out)             (read)
+ *   lse   [batch, hq, seqlen] fp32: the forward's lse (natural log)  (read)
+ *   dq    [batch, seqlen, hq, head_dim] dtype                        (written)
+ *   dk, dv [batch, seqlen, hkv, head_dim] dtype                      (written)
+ *   ws    >= moba_attn_bwd_workspace_size bytes of device scratch; its first
+ *         int32 is a status word (0) like the forward's.
+ * Every element of dq, dk, dv is written once (no atomics), so for one gate
+ * index (sel/offsets/rows) the gradients are bitwise reproducible; dk and dv
+ * sum over a group's rows in the order of `rows`. */
+MOBA_API moba_status_t moba_attn_bwd(const moba_shape_t* shape, const void* q, const void* k,
+                                     const void* v, const void* out, const void* dout, const float* lse,
+                                     const int32_t* sel, const int32_t* offsets, const int32_t* rows,
+                                     void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                     moba_stream_t stream);
+
 /* ---- the whole layer from host buffers ---------------------------------- */
 
 /* Device bytes moba_prefill_host needs for `shape` (with_lse: whether an lse

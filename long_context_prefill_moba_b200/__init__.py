@@ -32,6 +32,7 @@ __all__ = [
     "moba_attn_workspace_size", "moba_block_meanpool", "moba_gate_topk", "moba_attn_fwd",
     "moba_status_string", "moba_last_launch_count", "moba_gate_topk_noalloc", "MobaLayer", "moba_forward",
     "moba_prefill_host_workspace_size", "moba_prefill_host", "MobaHostLayer",
+    "moba_attn_bwd_workspace_size", "moba_attn_bwd",
     "MOBA_BF16", "MOBA_F32", "EXPORTED_SYMBOLS",
 ]
 
@@ -47,7 +48,8 @@ EXPORTED_SYMBOLS = [
     "moba_gate_workspace_size", "moba_attn_workspace_size", "moba_block_meanpool",
     "moba_gate_topk", "moba_attn_fwd", "moba_status_string", "moba_last_cuda_error",
     "moba_last_launch_count", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait",
-    "moba_prefill_host_workspace_size", "moba_prefill_host",
+    "moba_prefill_host_workspace_size", "moba_prefill_host", "moba_attn_bwd_workspace_size",
+    "moba_attn_bwd",
 ]
 
 
@@ -105,6 +107,10 @@ def load_library(path: str = LIB_PATH):
     L.moba_selftest_bounded_wait.restype = st
     L.moba_gate_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
     L.moba_gate_topk_noalloc.restype = st
+    L.moba_attn_bwd_workspace_size.argtypes = [P]
+    L.moba_attn_bwd_workspace_size.restype = sz
+    L.moba_attn_bwd.argtypes = [P] + [vp] * 13 + [sz, vp]
+    L.moba_attn_bwd.restype = st
     L.moba_prefill_host_workspace_size.argtypes = [P, st]
     L.moba_prefill_host_workspace_size.restype = sz
     L.moba_prefill_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -218,6 +224,17 @@ def moba_prefill_host(shape, q, k, v, out, lse, status, ws, stream=None):
            "moba_prefill_host")
 
 
+def moba_attn_bwd_workspace_size(shape) -> int:
+    return lib().moba_attn_bwd_workspace_size(_s(shape))
+
+
+def moba_attn_bwd(shape, q, k, v, out, dout, lse, sel, offsets, rows, dq, dk, dv, ws, stream=None):
+    _check(lib().moba_attn_bwd(_s(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                               _ptr(sel), _ptr(offsets), _ptr(rows), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moba_attn_bwd")
+
+
 class MobaHostLayer:
     """One MoBA layer shape served from host buffers (moba_prefill_host): the
     device workspace is allocated once; ``forward`` enqueues the copies and the
@@ -291,6 +308,18 @@ class MobaLayer:
         n += moba_last_launch_count()
         self.launches = n
         return out
+
+    def backward(self, q, k, v, out, lse, dout, dq, dk, dv, stream=None):
+        """dq, dk, dv of the last forward's attention given dout (the gate's
+        selection, sel/offsets/rows of that forward, is held fixed); `out` and
+        `lse` are that forward's outputs."""
+        if getattr(self, "bwd_ws", None) is None:
+            self.bwd_ws = torch.empty(moba_attn_bwd_workspace_size(self.shape), dtype=torch.uint8,
+                                      device=self.device)
+        moba_attn_bwd(self.shape, q, k, v, out, dout, lse, self.sel, self.offsets, self.rows, dq, dk, dv,
+                      self.bwd_ws, stream)
+        self.launches = moba_last_launch_count()
+        return dq, dk, dv
 
     def device_status(self):
         """(gate, attention) device status words of the last forward (synchronises):

@@ -250,6 +250,38 @@ MOBA_API moba_status_t moba_gate_topk_noalloc(const moba_shape_t* s, const void*
   return finish(e, launches);
 }
 
+MOBA_API size_t moba_attn_bwd_workspace_size(const moba_shape_t* s) {
+  if (moba_check_shape(s) != MOBA_OK) return 0;
+  return 256 + align_up((size_t)s->batch * s->seqlen * s->hq * sizeof(float));
+}
+
+MOBA_API moba_status_t moba_attn_bwd(const moba_shape_t* s, const void* q, const void* k, const void* v,
+                                     const void* out, const void* dout, const float* lse,
+                                     const int32_t* sel, const int32_t* offsets, const int32_t* rows,
+                                     void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                     moba_stream_t stream) {
+  g_last_launches = 0;
+  moba_status_t st = moba_check_shape(s);
+  if (st != MOBA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || dout == nullptr ||
+      lse == nullptr || sel == nullptr || offsets == nullptr || dq == nullptr || dk == nullptr ||
+      dv == nullptr || ws == nullptr)
+    return MOBA_ERR_INVALID_ARG;
+  if (rows == nullptr && rows_total(s) > 0) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned4(lse) || !aligned4(sel) || !aligned4(offsets) || (rows != nullptr && !aligned4(rows)) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(ws))
+    return MOBA_ERR_INVALID_ARG;
+  if (ws_bytes < moba_attn_bwd_workspace_size(s)) return MOBA_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  int launches = 0;
+  cudaError_t e = cudaMemsetAsync(base, 0, sizeof(int), (cudaStream_t)stream);
+  if (e == cudaSuccess)
+    e = moba::launch_attn_bwd(make_dims(s), s->dtype, q, k, v, out, dout, lse, sel, offsets, rows, dq, dk,
+                              dv, reinterpret_cast<float*>(base + 256), (cudaStream_t)stream, &launches);
+  return finish(e, launches);
+}
+
 MOBA_API size_t moba_prefill_host_workspace_size(const moba_shape_t* s, int with_lse) {
   if (moba_check_shape(s) != MOBA_OK) return 0;
   return host_layout(s, with_lse != 0).total;

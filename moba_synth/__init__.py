@@ -38,10 +38,11 @@ import torch
 
 __all__ = [
     "MobaConfig", "CONFIGS", "get_config", "normal_table",
-    "gen_q", "gen_k", "gen_v", "gen_rows", "TENSOR_Q", "TENSOR_K", "TENSOR_V", "TENSOR_OFF",
+    "gen_q", "gen_k", "gen_v", "gen_dout", "gen_rows", "TENSOR_Q", "TENSOR_K", "TENSOR_V", "TENSOR_OFF",
+    "TENSOR_DOUT",
 ]
 
-TENSOR_Q, TENSOR_K, TENSOR_V, TENSOR_OFF = 1, 2, 3, 4
+TENSOR_Q, TENSOR_K, TENSOR_V, TENSOR_OFF, TENSOR_DOUT = 1, 2, 3, 4, 5
 _M32 = 0xFFFFFFFF
 _MUL = 0x45D9F3B          # < 2^27, so (x < 2^32) * _MUL < 2^59: no int64 overflow
 _CHUNK = 1 << 25          # elements per generation chunk (bounds int64 temporaries)
@@ -164,6 +165,14 @@ def gen_v(cfg: MobaConfig, device="cpu") -> torch.Tensor:
     n = cfg.batch * cfg.seqlen * cfg.hkv * cfg.head_dim
     x = _flat_normals(0, n, cfg.seed, TENSOR_V, device)
     return _finish(x, cfg).view(cfg.batch, cfg.seqlen, cfg.hkv, cfg.head_dim)
+
+
+def gen_dout(cfg: MobaConfig, device="cpu") -> torch.Tensor:
+    """An upstream gradient dL/d(out), [batch, seqlen, hq, head_dim] in the
+    config dtype: standard normals of its own stream."""
+    n = cfg.batch * cfg.seqlen * cfg.hq * cfg.head_dim
+    x = _flat_normals(0, n, cfg.seed, TENSOR_DOUT, device)
+    return _finish(x, cfg).view(cfg.batch, cfg.seqlen, cfg.hq, cfg.head_dim)
 
 
 def _key_offsets(cfg: MobaConfig, device) -> torch.Tensor:
