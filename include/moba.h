@@ -203,9 +203,11 @@ MOBA_API size_t moba_attn_bwd_workspace_size(const moba_shape_t* shape);
  *   dk, dv [batch, seqlen, hkv, head_dim] dtype                      (written)
  *   ws    >= moba_attn_bwd_workspace_size bytes of device scratch; its first
  *         int32 is a status word (0) like the forward's.
- * Every element of dq, dk, dv is written once (no atomics), so for one gate
- * index (sel/offsets/rows) the gradients are bitwise reproducible; dk and dv
- * sum over a group's rows in the order of `rows`. */
+ * dk and dv are written once per key (for one gate index they are bitwise
+ * reproducible; they sum over a group's rows in the order of `rows`).  bf16
+ * with head_dim 128 runs on tensor cores and accumulates dq in fp32 with one
+ * vector reduction per row and selected block, so its last fp32 bits may
+ * depend on the order in which blocks arrive; the other layers write dq once. */
 MOBA_API moba_status_t moba_attn_bwd(const moba_shape_t* shape, const void* q, const void* k,
                                      const void* v, const void* out, const void* dout, const float* lse,
                                      const int32_t* sel, const int32_t* offsets, const int32_t* rows,

@@ -15,7 +15,9 @@
 //
 // Three launches: bwd_delta (D_r), bwd_dq (one warp per query row), bwd_dkv
 // (one warp per key).  Every output element is written once (no atomics), so
-// for one gate index the result is bitwise reproducible.
+// for one gate index the result is bitwise reproducible.  bf16 layers with
+// head_dim 128 run the tensor-core kernels of attn_bwd_tc.cu instead (after
+// the same bwd_delta).
 #include "launch.h"
 
 namespace moba {
@@ -222,19 +224,72 @@ cudaError_t launch_all(const Dims& dm, const void* q, const void* k, const void*
 
 }  // namespace
 
+__global__ void attn_plan_kernel(const int32_t* __restrict__ offsets, int ngroups, int tm,
+                                 int32_t* __restrict__ tile_start);
+int attn_bwd_tc_rows_per_tile();
+cudaError_t launch_bwd_kv_tc(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
+                             const float* lse, const float* delta, const int32_t* offsets, const int32_t* rows,
+                             void* dk, void* dv, int* status, cudaStream_t stream);
+cudaError_t launch_bwd_q_tc(const Dims& dm, bool cur, const void* q, const void* k, const void* v,
+                            const void* dout, const float* lse, const float* delta, const int32_t* offsets,
+                            const int32_t* rows, const int32_t* tile_start, float* dqacc, int* status, int ch,
+                            int64_t grid, cudaStream_t stream);
+cudaError_t launch_dq_convert(const float* acc, void* dq, int64_t n, cudaStream_t stream);
+
+bool attn_bwd_tc_path(const Dims& dm, int dtype) { return dtype == MOBA_BF16 && dm.d == 128; }
+
 cudaError_t launch_attn_bwd(const Dims& dm, int dtype, const void* q, const void* k, const void* v,
                             const void* out, const void* dout, const float* lse, const int32_t* sel,
                             const int32_t* offsets, const int32_t* rows, void* dq, void* dk, void* dv,
-                            float* delta, cudaStream_t stream, int* launches) {
+                            BwdWs ws, cudaStream_t stream, int* launches) {
+  if (attn_bwd_tc_path(dm, dtype)) {
+    const int64_t nrows = (int64_t)dm.batch * dm.N * dm.hq;
+    cudaError_t e = cudaMemsetAsync(ws.dqacc, 0, sizeof(float) * nrows * dm.d, stream);
+    if (e != cudaSuccess) return e;
+    bwd_delta_kernel<__nv_bfloat16, 128><<<(nrows + kWarps - 1) / kWarps, kWarps * 32, 0, stream>>>(
+        (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, ws.delta, nrows);
+    ++*launches;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // dk, dv: one CTA per 128-key tile
+    e = launch_bwd_kv_tc(dm, q, k, v, dout, lse, ws.delta, offsets, rows, dk, dv, ws.status, stream);
+    ++*launches;
+    if (e != cudaSuccess) return e;
+    // dq of the routed rows, pass by pass (row tiles of one gate group), then of the own block
+    const int KH = dm.topk - 1;
+    const int ngroups = dm.batch * dm.hkv * dm.n;
+    const int tm = attn_bwd_tc_rows_per_tile();
+    for (int ch = 0; ch < dm.nchunks && KH > 0; ++ch) {
+      const int t0 = ch * dm.chunk;
+      const int t1 = dm.N < t0 + dm.chunk ? dm.N : t0 + dm.chunk;
+      const int64_t nr = hist_rows_range(t0, t1, dm.B, KH) * dm.batch * dm.hq;
+      if (nr == 0) continue;
+      attn_plan_kernel<<<1, 1024, 0, stream>>>(offsets + (size_t)ch * ngroups, ngroups, tm, ws.tile_start);
+      ++*launches;
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      const int cmax = (t1 - 1) / dm.B;
+      const int64_t active = (int64_t)dm.batch * dm.hkv * (cmax < dm.n ? cmax : dm.n);
+      e = launch_bwd_q_tc(dm, false, q, k, v, dout, lse, ws.delta, offsets, rows, ws.tile_start, ws.dqacc,
+                          ws.status, ch, nr / tm + active + 1, stream);
+      ++*launches;
+      if (e != cudaSuccess) return e;
+    }
+    e = launch_bwd_q_tc(dm, true, q, k, v, dout, lse, ws.delta, offsets, rows, ws.tile_start, ws.dqacc,
+                        ws.status, 0, 0, stream);
+    ++*launches;
+    if (e != cudaSuccess) return e;
+    e = launch_dq_convert(ws.dqacc, dq, nrows * dm.d, stream);
+    ++*launches;
+    return e;
+  }
   if (dtype == MOBA_BF16)
     return dm.d == 128 ? launch_all<__nv_bfloat16, 128>(dm, q, k, v, out, dout, lse, sel, offsets, rows, dq,
-                                                        dk, dv, delta, stream, launches)
+                                                        dk, dv, ws.delta, stream, launches)
                        : launch_all<__nv_bfloat16, 64>(dm, q, k, v, out, dout, lse, sel, offsets, rows, dq,
-                                                       dk, dv, delta, stream, launches);
+                                                       dk, dv, ws.delta, stream, launches);
   return dm.d == 128 ? launch_all<float, 128>(dm, q, k, v, out, dout, lse, sel, offsets, rows, dq, dk, dv,
-                                              delta, stream, launches)
+                                              ws.delta, stream, launches)
                      : launch_all<float, 64>(dm, q, k, v, out, dout, lse, sel, offsets, rows, dq, dk, dv,
-                                             delta, stream, launches);
+                                             ws.delta, stream, launches);
 }
 
 }  // namespace moba

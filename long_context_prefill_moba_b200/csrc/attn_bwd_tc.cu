@@ -1,0 +1,619 @@
+// Backward of the attention step on 5th-generation tensor cores (bf16,
+// head_dim 128): the gradients of Softmax(q K[I]^T) V[I] ("MoBA: Mixture of
+// Block Attention for Long-Context LLMs", paper-graph summary §3 "The Core MoBA
+// Attention Equation", "Causality Enforcement"; Implementation, Algorithm 1
+// Steps 2-3 for the grouping of query rows by the block they attend) with the
+// gate's selection held fixed.  With the forward's lse L_r and
+// D_r = <dout_r, out_r>, for a tile of rows against a tile of keys:
+//   S = Q K^T, dP = dO V^T, P = exp(scale S - L), dS = P (dP - D),
+//   dV += P^T dO, dK += scale dS^T Q, dQ += scale dS K.
+// P needs no row max (the forward's L normalises it), so every element of a
+// tile is independent and the softmax warps split the key columns freely.
+//
+// bwd_kv_tc_kernel: one CTA per 128-key tile of one (b, kv head g, block j).
+//   dK and dV accumulate in TMEM over every query row that attends the tile:
+//   the rows the gate routed to block j in every pass (gathered through
+//   `rows`) and the rows of block j itself at or after the tile (causal, all G
+//   query heads).  Per 128-row tile: S and dP (SS MMAs), P and dS as bf16 into
+//   shared memory, dV += P^T dO and dK += dS^T Q (SS MMAs with A read
+//   MN-major).  Each key's dk, dv is written once.
+// bwd_q_tc_kernel: one CTA per 128-row tile, like the forward: kHist takes up
+//   to 128 rows of one gate group against all keys of block j, kCur 128
+//   tokens of one head against its own block (causal).  Per 128-key tile: S and
+//   dP, dS as bf16 into TMEM, dQ += dS K (TS MMA, K read MN-major).  The row
+//   tile's dQ is added into an fp32 accumulator with one vector reduction per
+//   row and 16 bytes (a row receives one per selected block).
+//
+// Every mbarrier wait is bounded (2 s); on expiry the CTA drains what it
+// issued, frees TMEM and writes MOBA_ERR_TIMEOUT to the status word.
+#include <cudaTypedefs.h>
+
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace moba {
+
+bool make_kv_map(CUtensorMap* map, const void* base, const Dims& dm);
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kT = 128;                     // rows or keys per tile
+constexpr uint32_t kTile = kT * kD * 2;     // 32 KB: two 16 KB column halves, 128-byte swizzle
+constexpr uint32_t kHalf = 16384;
+constexpr int kSoftmaxWarps = 8;
+
+MOBA_DEV uint32_t bar(const uint64_t* b) { return smem_u32(b); }
+
+MOBA_DEV void red_add_v4(float* dst, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+MOBA_DEV void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+// row r of q / dout (this warp's 64-column half) into the swizzled tile
+MOBA_DEV void load_half_row(uint32_t tile, int rho, int hf, const __nv_bfloat16* src, bool valid) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) cp_async16(tile + hf * kHalf + sw128_off(rho, c), src + hf * 64 + c * 8, valid);
+}
+
+// P or dS of one row and 64 keys (32 bf16 pairs) into a [row][key] tile read
+// MN-major as the A operand (M = keys, K = rows)
+MOBA_DEV void store_pairs(uint32_t tile, int rho, int hf, const uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    st_shared_v4(tile + hf * kHalf + sw128_off(rho, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+}
+
+// ============================================================================ dK, dV
+constexpr int kKvThreads = (kSoftmaxWarps + 1) * 32;
+constexpr uint32_t kKvOffK = 0, kKvOffV = kTile, kKvOffQ = 2 * kTile, kKvOffDO = 3 * kTile,
+                   kKvOffP = 4 * kTile, kKvOffDS = 5 * kTile;
+constexpr uint32_t kKvSmem = 6 * kTile + 1024;
+
+struct KvCtl {
+  uint64_t kv_full, q_full, s_full, p_full, mm_done, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// the query rows of row tile i of this key tile: the gate's groups of block j
+// over all passes, then block j's own tokens from the tile on, per query head
+struct RowTile {
+  bool own;          // block j's own rows (causal) or routed rows
+  int r0, cnt;       // routed: rows[r0 .. r0 + cnt)
+  int t0, h;         // own: tokens t0 .. t0 + 127 of head h
+};
+
+MOBA_DEV int kv_tiles(const int32_t* offsets, const Dims& dm, int b, int g, int j, int key0, int key_end,
+                      int& hist_tiles) {
+  const int64_t ngroups = (int64_t)dm.batch * dm.hkv * dm.n;
+  hist_tiles = 0;
+  for (int ch = 0; ch < dm.nchunks; ++ch) {
+    const int64_t gi = ch * ngroups + ((int64_t)b * dm.hkv + g) * dm.n + j;
+    hist_tiles += (offsets[gi + 1] - offsets[gi] + kT - 1) / kT;
+  }
+  return hist_tiles + (key_end - key0 + kT - 1) / kT * dm.G;
+}
+
+MOBA_DEV RowTile kv_row_tile(int i, int hist_tiles, const int32_t* offsets, const Dims& dm, int b, int g, int j,
+                             int key0) {
+  RowTile rt{};
+  if (i < hist_tiles) {
+    const int64_t ngroups = (int64_t)dm.batch * dm.hkv * dm.n;
+    int left = i;
+    for (int ch = 0; ch < dm.nchunks; ++ch) {
+      const int64_t gi = ch * ngroups + ((int64_t)b * dm.hkv + g) * dm.n + j;
+      const int r0 = offsets[gi], n = offsets[gi + 1] - r0;
+      const int nt = (n + kT - 1) / kT;
+      if (left < nt) {
+        rt.own = false;
+        rt.r0 = r0 + left * kT;
+        rt.cnt = min(kT, n - left * kT);
+        return rt;
+      }
+      left -= nt;
+    }
+  }
+  const int k = i - hist_tiles;
+  rt.own = true;
+  rt.t0 = key0 + (k / dm.G) * kT;
+  rt.h = g * dm.G + k % dm.G;
+  return rt;
+}
+
+__global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
+    const float* __restrict__ lse, const float* __restrict__ delta, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ rows, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+    int* __restrict__ status, Dims dm) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ KvCtl ctl;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int tiles_per_block = (dm.B + kT - 1) / kT;
+  int idx = blockIdx.x;
+  const int kt = idx % tiles_per_block; idx /= tiles_per_block;
+  const int j = idx % dm.n; idx /= dm.n;
+  const int g = idx % dm.hkv;
+  const int b = idx / dm.hkv;
+  const int key0 = j * dm.B + kt * kT;
+  const int key_end = min(dm.N, (j + 1) * dm.B);
+  if (b >= dm.batch || key0 >= key_end) return;
+  int hist_tiles;
+  const int ntiles = kv_tiles(offsets, dm, b, g, j, key0, key_end, hist_tiles);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    mbar_init(bar(&ctl.kv_full), kSoftmaxWarps);
+    mbar_init(bar(&ctl.q_full), kSoftmaxWarps);
+    mbar_init(bar(&ctl.s_full), 1);
+    mbar_init(bar(&ctl.p_full), kSoftmaxWarps);
+    mbar_init(bar(&ctl.mm_done), 1);
+    mbar_init(bar(&ctl.drain), 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kSoftmaxWarps) {
+    tmem_alloc(smem_u32(&ctl.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = ctl.tmem_base;
+  volatile int* abort_flag = &ctl.abort;
+
+  if (warp < kSoftmaxWarps) {
+    const int qd = warp & 3, hf = warp >> 2;
+    const int rho = qd * 32 + lane;           // TMEM lane: a row of S/dP, a key of dK/dV
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    const float sl2 = dm.scale_log2;
+    {
+      const int u = key0 + rho;
+      const bool ok = u < key_end;
+      const size_t kr = ((size_t)b * dm.N + (ok ? u : 0)) * dm.hkv + g;
+      load_half_row(base + kKvOffK, rho, hf, k + kr * kD, ok);
+      load_half_row(base + kKvOffV, rho, hf, v + kr * kD, ok);
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(&ctl.kv_full));
+    }
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      if (i > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.mm_done), (i - 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      const RowTile rt = kv_row_tile(i, hist_tiles, offsets, dm, b, g, j, key0);
+      int r = 0, t = 0, h = 0;
+      bool valid;
+      if (rt.own) {
+        t = rt.t0 + rho;
+        h = rt.h;
+        valid = t < key_end;
+        r = (b * dm.N + t) * dm.hq + h;
+      } else {
+        valid = rho < rt.cnt;
+        r = valid ? rows[rt.r0 + rho] : 0;
+        h = r % dm.hq;
+        t = (r / dm.hq) % dm.N;
+      }
+      load_half_row(base + kKvOffQ, rho, hf, q + (size_t)(valid ? r : 0) * kD, valid);
+      load_half_row(base + kKvOffDO, rho, hf, dout + (size_t)(valid ? r : 0) * kD, valid);
+      const float L2 = valid ? lse[((size_t)b * dm.hq + h) * dm.N + t] * kLog2e : INFINITY;
+      const float Dr = valid ? delta[r] : 0.f;
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(&ctl.q_full));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.s_full), i & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[64], dr[64];
+      tmem_ld32(tb + 64u * hf + lane_off, sr);
+      tmem_ld32(tb + 64u * hf + 32 + lane_off, sr + 32);
+      tmem_ld32(tb + 128u + 64u * hf + lane_off, dr);
+      tmem_ld32(tb + 128u + 64u * hf + 32 + lane_off, dr + 32);
+      tmem_wait_ld();
+      // keys of this warp's half valid for the row: u < key_end, and u <= t in the own block
+      const int ulim = min(key_end, rt.own ? t + 1 : key_end) - (key0 + 64 * hf);   // keys [0, ulim)
+      uint32_t pp[32], ps[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        float p0 = exp2f(__uint_as_float(sr[2 * c]) * sl2 - L2);
+        float p1 = exp2f(__uint_as_float(sr[2 * c + 1]) * sl2 - L2);
+        p0 = 2 * c < ulim ? p0 : 0.f;
+        p1 = 2 * c + 1 < ulim ? p1 : 0.f;
+        pp[c] = pack_bf16x2(p0, p1);
+        ps[c] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * c]) - Dr), p1 * (__uint_as_float(dr[2 * c + 1]) - Dr));
+      }
+      store_pairs(base + kKvOffP, rho, hf, pp);
+      store_pairs(base + kKvOffDS, rho, hf, ps);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(&ctl.p_full));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.mm_done), (ntiles - 1) & 1, abort_flag));
+    if (ok) {
+      // dK, dV rows (lanes = keys) of this warp's 64 columns
+      tc_fence_after();
+      const int u = key0 + rho;
+      const float scale = sl2 / kLog2e;
+      const size_t kr = ((size_t)b * dm.N + u) * dm.hkv + g;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t gvv[32], gkk[32];
+        tmem_ld32(tb + 256u + 64u * hf + 32u * cc + lane_off, gvv);
+        tmem_ld32(tb + 384u + 64u * hf + 32u * cc + lane_off, gkk);
+        tmem_wait_ld();
+        if (u < key_end) {
+          uint4* dvp = reinterpret_cast<uint4*>(dv + kr * kD + 64 * hf + 32 * cc);
+          uint4* dkp = reinterpret_cast<uint4*>(dk + kr * kD + 64 * hf + 32 * cc);
+#pragma unroll
+          for (int e8 = 0; e8 < 4; ++e8) {
+            dvp[e8] = make_uint4(
+                pack_bf16x2(__uint_as_float(gvv[8 * e8 + 0]), __uint_as_float(gvv[8 * e8 + 1])),
+                pack_bf16x2(__uint_as_float(gvv[8 * e8 + 2]), __uint_as_float(gvv[8 * e8 + 3])),
+                pack_bf16x2(__uint_as_float(gvv[8 * e8 + 4]), __uint_as_float(gvv[8 * e8 + 5])),
+                pack_bf16x2(__uint_as_float(gvv[8 * e8 + 6]), __uint_as_float(gvv[8 * e8 + 7])));
+            dkp[e8] = make_uint4(
+                pack_bf16x2(__uint_as_float(gkk[8 * e8 + 0]) * scale, __uint_as_float(gkk[8 * e8 + 1]) * scale),
+                pack_bf16x2(__uint_as_float(gkk[8 * e8 + 2]) * scale, __uint_as_float(gkk[8 * e8 + 3]) * scale),
+                pack_bf16x2(__uint_as_float(gkk[8 * e8 + 4]) * scale, __uint_as_float(gkk[8 * e8 + 5]) * scale),
+                pack_bf16x2(__uint_as_float(gkk[8 * e8 + 6]) * scale, __uint_as_float(gkk[8 * e8 + 7]) * scale));
+          }
+        }
+      }
+    }
+  } else if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idS = idesc_bf16(128, kT, false);          // A, B K-major
+    const uint32_t idG = idesc_bf16_amn(128, kD, true);       // A, B MN-major
+    const uint32_t hi = sdesc_hi(1024);
+    const uint32_t loK = sdesc_lo(base + kKvOffK, 16), loV = sdesc_lo(base + kKvOffV, 16),
+                   loQ = sdesc_lo(base + kKvOffQ, 16), loDO = sdesc_lo(base + kKvOffDO, 16);
+    const uint32_t mnQ = sdesc_lo(base + kKvOffQ, kHalf), mnDO = sdesc_lo(base + kKvOffDO, kHalf),
+                   mnP = sdesc_lo(base + kKvOffP, kHalf), mnDS = sdesc_lo(base + kKvOffDS, kHalf);
+    bool ok = mbar_wait(bar(&ctl.kv_full), 0, abort_flag);
+    for (int i = 0; i < ntiles && ok; ++i) {
+      if (!(ok = mbar_wait(bar(&ctl.q_full), i & 1, abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+        mma_ss(tb, sdesc_join(loQ + off, hi), sdesc_join(loK + off, hi), idS, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+        mma_ss(tb + 128u, sdesc_join(loDO + off, hi), sdesc_join(loV + off, hi), idS, kk > 0);
+      }
+      mma_commit(bar(&ctl.s_full));
+      if (!(ok = mbar_wait(bar(&ctl.p_full), i & 1, abort_flag))) break;
+      tc_fence_after();
+      // dV += P^T dO and dK += dS^T Q: K runs over the 128 rows, 16 per MMA
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk * 2048) >> 4;
+        mma_ss(tb + 256u, sdesc_join(mnP + off, hi), sdesc_join(mnDO + off, hi), idG, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk * 2048) >> 4;
+        mma_ss(tb + 384u, sdesc_join(mnDS + off, hi), sdesc_join(mnQ + off, hi), idG, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(bar(&ctl.mm_done));
+    }
+    if (!ok) {
+      int never = 0;
+      mma_commit(bar(&ctl.drain));
+      mbar_wait(bar(&ctl.drain), 0, &never);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kSoftmaxWarps) tmem_dealloc(tb, 512);
+  if (tid == 0 && ctl.abort) atomicExch(status, (int)MOBA_ERR_TIMEOUT);
+}
+
+// ============================================================================ dQ
+constexpr int kHist = 0, kCur = 1;
+constexpr int kQThreads = (kSoftmaxWarps + 2) * 32;   // softmax, TMA producer, MMA issuer
+constexpr uint32_t kQOffQ = 0, kQOffDO = kTile, kQOffK = 2 * kTile, kQOffV = 4 * kTile;
+constexpr uint32_t kQSmem = 6 * kTile + 1024;
+
+struct QCtl {
+  uint64_t q_full, k_full[2], v_full[2], k_free[2], v_free[2], s_full, p_full, o_full, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kQThreads, 1) bwd_q_tc_kernel(
+    const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap tmK,
+    const __grid_constant__ CUtensorMap tmV, const __nv_bfloat16* __restrict__ dout,
+    const float* __restrict__ lse, const float* __restrict__ delta, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ rows, const int32_t* __restrict__ tile_start, float* __restrict__ dqacc,
+    int* __restrict__ status, Dims dm, int ch) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ QCtl ctl;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+
+  // ---- the row tile and its keys
+  int b, g, key0, nkt, r0 = 0, cnt = 0, t_first = 0, h_cur = 0;
+  if (MODE == kHist) {
+    const int ngroups = dm.batch * dm.hkv * dm.n;
+    const int tile = blockIdx.x;
+    if (tile >= tile_start[ngroups]) return;
+    int lo = 0, hi = ngroups - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tile_start[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int j = lo % dm.n;
+    g = (lo / dm.n) % dm.hkv;
+    b = lo / (dm.n * dm.hkv);
+    const size_t goff = (size_t)ch * ngroups + lo;
+    r0 = offsets[goff] + (tile - tile_start[lo]) * kT;
+    cnt = min(kT, offsets[goff + 1] - r0);
+    key0 = j * dm.B;
+    nkt = (dm.B + kT - 1) / kT;
+  } else {
+    const int ntile = (dm.N + kT - 1) / kT;
+    int idx = blockIdx.x;
+    const int tau = idx % ntile; idx /= ntile;
+    h_cur = idx % dm.hq;
+    b = idx / dm.hq;
+    if (b >= dm.batch) return;
+    g = h_cur / dm.G;
+    t_first = tau * kT;
+    const int t_last = min(dm.N, t_first + kT) - 1;
+    key0 = (t_first / dm.B) * dm.B;
+    nkt = (t_last - key0) / kT + 1;
+  }
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    mbar_init(bar(&ctl.q_full), kSoftmaxWarps);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(&ctl.k_full[s]), 1);
+      mbar_init(bar(&ctl.v_full[s]), 1);
+      mbar_init(bar(&ctl.k_free[s]), 1);
+      mbar_init(bar(&ctl.v_free[s]), 1);
+    }
+    mbar_init(bar(&ctl.s_full), 1);
+    mbar_init(bar(&ctl.p_full), kSoftmaxWarps);
+    mbar_init(bar(&ctl.o_full), 1);
+    mbar_init(bar(&ctl.drain), 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kSoftmaxWarps) {
+    tmem_alloc(smem_u32(&ctl.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = ctl.tmem_base;
+  volatile int* abort_flag = &ctl.abort;
+
+  if (warp < kSoftmaxWarps) {
+    const int qd = warp & 3, hf = warp >> 2;
+    const int rho = qd * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    const float sl2 = dm.scale_log2;
+    bool valid;
+    int r, t, h;
+    if (MODE == kHist) {
+      valid = rho < cnt;
+      r = valid ? rows[r0 + rho] : 0;
+      h = r % dm.hq;
+      t = (r / dm.hq) % dm.N;
+    } else {
+      t = t_first + rho;
+      valid = t < dm.N;
+      h = h_cur;
+      r = valid ? (b * dm.N + t) * dm.hq + h : 0;
+    }
+    load_half_row(base + kQOffQ, rho, hf, q + (size_t)r * kD, valid);
+    load_half_row(base + kQOffDO, rho, hf, dout + (size_t)r * kD, valid);
+    const float L2 = valid ? lse[((size_t)b * dm.hq + h) * dm.N + t] * kLog2e : INFINITY;
+    const float Dr = valid ? delta[r] : 0.f;
+    cp_async_commit();
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(&ctl.q_full));
+    // keys valid for the row: [lo_u, hi_u]
+    const int lo_u = MODE == kHist ? key0 : (t / dm.B) * dm.B;
+    const int hi_u = MODE == kHist ? min(dm.N, key0 + dm.B) - 1 : t;
+    bool ok = true;
+    for (int i = 0; i < nkt && ok; ++i) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.s_full), i & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[64], dr[64];
+      tmem_ld32(tb + 64u * hf + lane_off, sr);
+      tmem_ld32(tb + 64u * hf + 32 + lane_off, sr + 32);
+      tmem_ld32(tb + 128u + 64u * hf + lane_off, dr);
+      tmem_ld32(tb + 128u + 64u * hf + 32 + lane_off, dr + 32);
+      tmem_wait_ld();
+      const int u0 = key0 + i * kT + 64 * hf;     // key of column 0 of this warp's half
+      const int vlo = lo_u - u0, vhi = hi_u - u0;
+      uint32_t ps[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        float p0 = exp2f(__uint_as_float(sr[2 * c]) * sl2 - L2);
+        float p1 = exp2f(__uint_as_float(sr[2 * c + 1]) * sl2 - L2);
+        p0 = (2 * c >= vlo && 2 * c <= vhi) ? p0 : 0.f;
+        p1 = (2 * c + 1 >= vlo && 2 * c + 1 <= vhi) ? p1 : 0.f;
+        ps[c] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * c]) - Dr), p1 * (__uint_as_float(dr[2 * c + 1]) - Dr));
+      }
+      // dS over this warp's own dP columns [64 hf, 64 hf + 32): already read
+      tmem_st32(tb + 128u + 64u * hf + lane_off, ps);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(&ctl.p_full));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.o_full), 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      const float scale = sl2 / kLog2e;
+      float* dst = dqacc + (size_t)r * kD + 64 * hf;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tb + 256u + 64u * hf + 32u * cc + lane_off, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4)
+            red_add_v4(dst + 32 * cc + 4 * e4, __uint_as_float(o[4 * e4]) * scale,
+                       __uint_as_float(o[4 * e4 + 1]) * scale, __uint_as_float(o[4 * e4 + 2]) * scale,
+                       __uint_as_float(o[4 * e4 + 3]) * scale);
+        }
+      }
+    }
+  } else if (warp == kSoftmaxWarps) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const int y0 = b * dm.N + key0;
+      const int x0 = g * kD;
+      int issued_k = 0, issued_v = 0;
+      for (int i = 0; i < nkt; ++i) {
+        const int s = i & 1;
+        const uint32_t ks = base + kQOffK + s * kTile, vs = base + kQOffV + s * kTile;
+        if (i >= 2 && !mbar_wait(bar(&ctl.k_free[s]), ((i >> 1) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(&ctl.k_full[s]), kTile);
+        tma_load_2d(ks, &tmK, x0, y0 + i * kT, bar(&ctl.k_full[s]));
+        tma_load_2d(ks + kHalf, &tmK, x0 + 64, y0 + i * kT, bar(&ctl.k_full[s]));
+        issued_k = i + 1;
+        if (i >= 2 && !mbar_wait(bar(&ctl.v_free[s]), ((i >> 1) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(&ctl.v_full[s]), kTile);
+        tma_load_2d(vs, &tmV, x0, y0 + i * kT, bar(&ctl.v_full[s]));
+        tma_load_2d(vs + kHalf, &tmV, x0 + 64, y0 + i * kT, bar(&ctl.v_full[s]));
+        issued_v = i + 1;
+      }
+      if (*abort_flag) {
+        int never = 0;
+        for (int i = (issued_k > 2 ? issued_k - 2 : 0); i < issued_k; ++i)
+          mbar_wait(bar(&ctl.k_full[i & 1]), (i >> 1) & 1, &never);
+        for (int i = (issued_v > 2 ? issued_v - 2 : 0); i < issued_v; ++i)
+          mbar_wait(bar(&ctl.v_full[i & 1]), (i >> 1) & 1, &never);
+      }
+    }
+  } else if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idS = idesc_bf16(128, kT, false);
+    const uint32_t idQ = idesc_bf16(128, kD, true);        // B (K tile) read MN-major
+    const uint32_t hi = sdesc_hi(1024);
+    const uint32_t loQ = sdesc_lo(base + kQOffQ, 16), loDO = sdesc_lo(base + kQOffDO, 16),
+                   loK = sdesc_lo(base + kQOffK, 16), loV = sdesc_lo(base + kQOffV, 16),
+                   mnK = sdesc_lo(base + kQOffK, kHalf);
+    bool ok = mbar_wait(bar(&ctl.q_full), 0, abort_flag);
+    for (int i = 0; i < nkt && ok; ++i) {
+      const int s = i & 1;
+      ok = mbar_wait(bar(&ctl.k_full[s]), (i >> 1) & 1, abort_flag) &&
+           mbar_wait(bar(&ctl.v_full[s]), (i >> 1) & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t ko = s ? (kTile >> 4) : 0u;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+        mma_ss(tb, sdesc_join(loQ + off, hi), sdesc_join(loK + ko + off, hi), idS, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+        mma_ss(tb + 128u, sdesc_join(loDO + off, hi), sdesc_join(loV + ko + off, hi), idS, kk > 0);
+      }
+      mma_commit(bar(&ctl.s_full));
+      mma_commit(bar(&ctl.v_free[s]));
+      if (!(ok = mbar_wait(bar(&ctl.p_full), i & 1, abort_flag))) break;
+      tc_fence_after();
+      // dQ += dS K: dS of keys 0-63 in columns 128-159, keys 64-127 in 192-223
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t a = tb + 128u + (kk < 4 ? kk * 8u : 64u + (kk - 4) * 8u);
+        mma_ts(tb + 256u, a, sdesc_join(mnK + ko + ((kk * 2048) >> 4), hi), idQ, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(bar(&ctl.k_free[s]));
+    }
+    if (ok) {
+      mma_commit(bar(&ctl.o_full));
+    } else {
+      int never = 0;
+      mma_commit(bar(&ctl.drain));
+      mbar_wait(bar(&ctl.drain), 0, &never);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kSoftmaxWarps) tmem_dealloc(tb, 512);
+  if (tid == 0 && ctl.abort) atomicExch(status, (int)MOBA_ERR_TIMEOUT);
+}
+
+__global__ void dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, int64_t n4) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 x = reinterpret_cast<const float4*>(acc)[i];
+  reinterpret_cast<uint2*>(dq)[i] = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+}
+
+}  // namespace
+
+int attn_bwd_tc_rows_per_tile() { return kT; }
+
+cudaError_t launch_bwd_kv_tc(const Dims& dm, const void* q, const void* k, const void* v, const void* dout,
+                             const float* lse, const float* delta, const int32_t* offsets, const int32_t* rows,
+                             void* dk, void* dv, int* status, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(bwd_kv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = (int64_t)dm.batch * dm.hkv * dm.n * ((dm.B + kT - 1) / kT);
+  bwd_kv_tc_kernel<<<grid, kKvThreads, kKvSmem, stream>>>(
+      (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, (const __nv_bfloat16*)dout,
+      lse, delta, offsets, rows, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, status, dm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_q_tc(const Dims& dm, bool cur, const void* q, const void* k, const void* v,
+                            const void* dout, const float* lse, const float* delta, const int32_t* offsets,
+                            const int32_t* rows, const int32_t* tile_start, float* dqacc, int* status, int ch,
+                            int64_t grid, cudaStream_t stream) {
+  CUtensorMap mk, mv;
+  if (!make_kv_map(&mk, k, dm) || !make_kv_map(&mv, v, dm)) return cudaErrorInvalidValue;
+  auto kern = cur ? bwd_q_tc_kernel<kCur> : bwd_q_tc_kernel<kHist>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
+  if (e != cudaSuccess) return e;
+  if (cur) grid = (int64_t)((dm.N + kT - 1) / kT) * dm.hq * dm.batch;
+  kern<<<grid, kQThreads, kQSmem, stream>>>((const __nv_bfloat16*)q, mk, mv, (const __nv_bfloat16*)dout, lse,
+                                            delta, offsets, rows, tile_start, dqacc, status, dm, ch);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dq_convert(const float* acc, void* dq, int64_t n, cudaStream_t stream) {
+  const int64_t n4 = n / 4;
+  dq_convert_kernel<<<(n4 + 255) / 256, 256, 0, stream>>>(acc, (__nv_bfloat16*)dq, n4);
+  return cudaGetLastError();
+}
+
+}  // namespace moba

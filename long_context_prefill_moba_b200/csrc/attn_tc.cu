@@ -576,6 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   if (tid == 0 && ctl.abort) atomicExch(status, (int)MOBA_ERR_TIMEOUT);
 }
 
+}  // namespace
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -601,6 +603,8 @@ bool make_kv_map(CUtensorMap* map, const void* base, const Dims& dm) {
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 // the setmaxnreg split is only safe if the kernel really launches with kLaunchRegs
 template <int MODE>

@@ -61,12 +61,18 @@ cudaError_t launch_attn_passes(const Dims& dm, int dtype, const void* q, const v
                                int ch_end, cudaStream_t stream, int* launches);
 
 // backward of the attention step: dq, dk, dv (in the input dtype) given dout,
-// the forward's out and lse and the gate's sel/offsets/rows; delta is
-// batch*seqlen*hq fp32 scratch
+// the forward's out and lse and the gate's sel/offsets/rows
+struct BwdWs {
+  int* status;          // device status word
+  float* delta;         // [b * N * hq]      <dout, out> per row
+  float* dqacc;         // [b * N * hq, d]   fp32 dq accumulator (tensor-core path)
+  int32_t* tile_start;  // [b * hkv * n + 1] row-tile prefix of one pass (tensor-core path)
+};
+bool attn_bwd_tc_path(const Dims& dm, int dtype);
 cudaError_t launch_attn_bwd(const Dims& dm, int dtype, const void* q, const void* k, const void* v,
                             const void* out, const void* dout, const float* lse, const int32_t* sel,
                             const int32_t* offsets, const int32_t* rows, void* dq, void* dk, void* dv,
-                            float* delta, cudaStream_t stream, int* launches);
+                            BwdWs ws, cudaStream_t stream, int* launches);
 
 // a kernel whose only wait can never complete: it must time out (status word)
 cudaError_t launch_bounded_wait_selftest(int* status, cudaStream_t stream);

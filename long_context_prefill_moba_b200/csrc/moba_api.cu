@@ -250,9 +250,24 @@ MOBA_API moba_status_t moba_gate_topk_noalloc(const moba_shape_t* s, const void*
   return finish(e, launches);
 }
 
+struct BwdLayout {
+  size_t status, delta, dqacc, tile_start, total;
+};
+BwdLayout bwd_layout(const moba_shape_t* s) {
+  const size_t nrows = (size_t)s->batch * s->seqlen * s->hq;
+  const bool tc = moba::attn_bwd_tc_path(make_dims(s), s->dtype);
+  BwdLayout L;
+  L.status = 0;
+  L.delta = 256;
+  L.dqacc = L.delta + align_up(nrows * sizeof(float));
+  L.tile_start = L.dqacc + (tc ? align_up(nrows * s->head_dim * sizeof(float)) : 0);
+  L.total = L.tile_start + (tc ? align_up(((size_t)s->batch * s->hkv * nblocks(s) + 1) * sizeof(int32_t)) : 0);
+  return L;
+}
+
 MOBA_API size_t moba_attn_bwd_workspace_size(const moba_shape_t* s) {
   if (moba_check_shape(s) != MOBA_OK) return 0;
-  return 256 + align_up((size_t)s->batch * s->seqlen * s->hq * sizeof(float));
+  return bwd_layout(s).total;
 }
 
 MOBA_API moba_status_t moba_attn_bwd(const moba_shape_t* s, const void* q, const void* k, const void* v,
@@ -274,11 +289,14 @@ MOBA_API moba_status_t moba_attn_bwd(const moba_shape_t* s, const void* q, const
     return MOBA_ERR_INVALID_ARG;
   if (ws_bytes < moba_attn_bwd_workspace_size(s)) return MOBA_ERR_WORKSPACE;
   char* base = static_cast<char*>(ws);
+  const BwdLayout L = bwd_layout(s);
+  moba::BwdWs w{reinterpret_cast<int*>(base + L.status), reinterpret_cast<float*>(base + L.delta),
+                reinterpret_cast<float*>(base + L.dqacc), reinterpret_cast<int32_t*>(base + L.tile_start)};
   int launches = 0;
-  cudaError_t e = cudaMemsetAsync(base, 0, sizeof(int), (cudaStream_t)stream);
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(int), (cudaStream_t)stream);
   if (e == cudaSuccess)
     e = moba::launch_attn_bwd(make_dims(s), s->dtype, q, k, v, out, dout, lse, sel, offsets, rows, dq, dk,
-                              dv, reinterpret_cast<float*>(base + 256), (cudaStream_t)stream, &launches);
+                              dv, w, (cudaStream_t)stream, &launches);
   return finish(e, launches);
 }
 

@@ -121,6 +121,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// the same with the A operand read MN-major from shared memory (bit 15)
+__host__ __device__ constexpr uint32_t idesc_bf16_amn(int M, int N, bool b_mn_major) {
+  return idesc_bf16(M, N, b_mn_major) | (1u << 15);
+}
 
 // Shared-memory matrix descriptor, 128-byte swizzle:
 // bits [0,14) start >> 4, [16,30) leading-dim byte offset >> 4,

@@ -24,6 +24,9 @@ CASES = {
     "f32_d128_multipass": (S.get_config("tiny").replace(batch=1, seqlen=600, hq=2, hkv=1, head_dim=128,
                                                         block=64, topk=5), 128),
     "f32_ragged_gqa": (S.get_config("tiny").replace(batch=2, seqlen=333, hq=4, hkv=2, block=40, topk=4), 0),
+    # tensor-core path with several row tiles per key tile and four passes
+    "bf16_multitile": (S.get_config("mqar").replace(batch=1, seqlen=4096, hq=8, hkv=2, block=512, topk=4),
+                       1024),
 }
 
 
@@ -50,19 +53,29 @@ def test_backward_parity(cuda_device, name):
     res, dq, dk, dv = run_backward(cfg, chunk)
     sel = res["layer"].sel_view().cpu().numpy()
     q, k, v, dout = S.gen_q(cfg), S.gen_k(cfg), S.gen_v(cfg), S.gen_dout(cfg)
-    rq, rk, rv, _ = OB.moba_backward(q, k, v, dout, cfg.block, cfg.topk, cfg.softmax_scale, sel=sel)
+    if cfg.seqlen > 2048:
+        # the dense-mask formulation (pinned against the gather one) is the fast one at this size
+        rq, rk, rv = OB.moba_backward_dense(q, k, v, dout, sel, cfg.block, cfg.softmax_scale)
+    else:
+        rq, rk, rv, _ = OB.moba_backward(q, k, v, dout, cfg.block, cfg.topk, cfg.softmax_scale, sel=sel)
     for name_, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
         err = float(np.abs(cpu(got).numpy() - ref).max())
         print(name, name_, "max abs err", err, "max |ref|", float(np.abs(ref).max()))
         assert err <= tol(cfg, ref), (name_, err)
 
 
-def test_backward_is_reproducible(cuda_device):
-    # no atomics: for one gate index the gradients are bitwise the same
-    cfg, chunk = CASES["ragged_multipass"]
+@pytest.mark.parametrize("name", ["ragged_multipass", "d64_bf16"])
+def test_backward_is_reproducible(cuda_device, name):
+    # dk, dv are written once per key: for one gate index they are bitwise the
+    # same; dq too on the CUDA-core path (d64), within rounding on tensor cores
+    cfg, chunk = CASES[name]
     res, dq1, dk1, dv1 = run_backward(cfg, chunk)
     dout = S.gen_dout(cfg, res["q"].device)
     dq2, dk2, dv2 = torch.empty_like(dq1), torch.empty_like(dk1), torch.empty_like(dv1)
     res["layer"].backward(res["q"], res["k"], res["v"], res["out"], res["lse"], dout, dq2, dk2, dv2)
     torch.cuda.synchronize()
-    assert torch.equal(dq1, dq2) and torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    if cfg.head_dim != 128:
+        assert torch.equal(dq1, dq2)
+    else:
+        assert (dq1.float() - dq2.float()).abs().max().item() <= 1e-2
