@@ -266,6 +266,43 @@ def config_of(cfg, args):
 # Speed-up curve: MoBA layer vs dense causal attention at growing lengths
 # (the comparison of the paper's Figure 2a, on this GPU)
 # ---------------------------------------------------------------------------
+def backward_bench(cfg, steps, warmup):
+    """One JSON line: the attention backward (moba_attn_bwd: dq, dk, dv given a
+    seeded dout, the gate's selection of the forward held fixed) on `cfg`,
+    inputs resident in HBM, CUDA events on the stream.  Algorithmic FLOPs are
+    2.5x the forward's (5 matrix products per attended pair: the score
+    recompute, dP, dV, dK, dQ); the tensor-core path also recomputes S and dP
+    once more for dQ, which is not counted."""
+    import long_context_prefill_moba_b200 as M
+    M.load_library()
+    dev = torch.device("cuda", 0)
+    q, k, v = S.gen_q(cfg, dev), S.gen_k(cfg, dev), S.gen_v(cfg, dev)
+    dout = S.gen_dout(cfg, dev)
+    layer = M.MobaLayer.from_config(cfg, dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(cfg.batch, cfg.hq, cfg.seqlen, dtype=torch.float32, device=dev)
+    layer.forward(q, k, v, out, lse)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for _ in range(warmup):
+        layer.backward(q, k, v, out, lse, dout, dq, dk, dv)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        layer.backward(q, k, v, out, lse, dout, dq, dk, dv)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    status = layer.bwd_ws[:4].view(torch.int32).item()
+    flops = 2.5 * attn_flops(cfg)
+    peaks, _ = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    print(json.dumps({"mode": "backward", "workload": cfg.name, "seqlen": cfg.seqlen, "ms_per_layer": ms,
+                      "tflops": flops / ms / 1e9, "frac_of_sustained_peak": flops / ms / 1e9 / peak,
+                      "steps": steps, "warmup": warmup, "gpu_launches_per_step": layer.launches,
+                      "device_status": status}), flush=True)
+
+
 def speedup_curve(seqlens, reps=2):
     """One JSON line per sequence length: the MoBA layer (mean-pool + gate +
     attention through the C ABI) against dense causal attention on the same
@@ -339,6 +376,8 @@ def main():
     ap.add_argument("--config", default="1m", choices=sorted(S.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--backward", action="store_true",
+                    help="time the attention backward (moba_attn_bwd) instead; prints its own JSON line")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
@@ -349,6 +388,9 @@ def main():
     args = ap.parse_args()
     if args.speedup_curve:
         speedup_curve([int(x) for x in args.curve_seqlens.split(",")])
+        return
+    if args.backward:
+        backward_bench(S.get_config(args.config), args.steps, args.warmup)
         return
     cfg = S.get_config(args.config)
 

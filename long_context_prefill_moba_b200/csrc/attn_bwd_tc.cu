@@ -14,9 +14,11 @@
 //   dK and dV accumulate in TMEM over every query row that attends the tile:
 //   the rows the gate routed to block j in every pass (gathered through
 //   `rows`) and the rows of block j itself at or after the tile (causal, all G
-//   query heads).  Per 128-row tile: S and dP (SS MMAs), P and dS as bf16 into
-//   shared memory, dV += P^T dO and dK += dS^T Q (SS MMAs with A read
-//   MN-major).  Each key's dk, dv is written once.
+//   query heads).  Per 128-row tile: S^T = K Q^T and dP^T = V dO^T (SS MMAs,
+//   a key per TMEM lane), P^T and dS^T as bf16 back into TMEM, dV += P^T dO
+//   and dK += dS^T Q (TS MMAs, dO and Q read MN-major); the next row tile's
+//   q/dout rows load into the second stage meanwhile.  Each key's dk, dv is
+//   written once.
 // bwd_q_tc_kernel: one CTA per 128-row tile, like the forward: kHist takes up
 //   to 128 rows of one gate group against all keys of block j, kCur 128
 //   tokens of one head against its own block (causal).  Per 128-key tile: S and
@@ -51,10 +53,6 @@ MOBA_DEV void red_add_v4(float* dst, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
-MOBA_DEV void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
 
 // row r of q / dout (this warp's 64-column half) into the swizzled tile
 MOBA_DEV void load_half_row(uint32_t tile, int rho, int hf, const __nv_bfloat16* src, bool valid) {
@@ -62,24 +60,22 @@ MOBA_DEV void load_half_row(uint32_t tile, int rho, int hf, const __nv_bfloat16*
   for (int c = 0; c < 8; ++c) cp_async16(tile + hf * kHalf + sw128_off(rho, c), src + hf * 64 + c * 8, valid);
 }
 
-// P or dS of one row and 64 keys (32 bf16 pairs) into a [row][key] tile read
-// MN-major as the A operand (M = keys, K = rows)
-MOBA_DEV void store_pairs(uint32_t tile, int rho, int hf, const uint32_t (&pk)[32]) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c)
-    st_shared_v4(tile + hf * kHalf + sw128_off(rho, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-}
-
 // ============================================================================ dK, dV
+// Transposed products: S^T = K Q^T and dP^T = V dO^T put a key on every TMEM
+// lane, so P^T and dS^T stay in TMEM as bf16 and feed dV += P^T dO and
+// dK += dS^T Q as TS MMAs; shared memory holds K, V and two Q/dO row tiles,
+// and the next row tile loads while the current one computes.
 constexpr int kKvThreads = (kSoftmaxWarps + 1) * 32;
-constexpr uint32_t kKvOffK = 0, kKvOffV = kTile, kKvOffQ = 2 * kTile, kKvOffDO = 3 * kTile,
-                   kKvOffP = 4 * kTile, kKvOffDS = 5 * kTile;
+constexpr uint32_t kKvOffK = 0, kKvOffV = kTile, kKvOffQ = 2 * kTile;   // Q/dO stage x at kKvOffQ + 2x kTile
 constexpr uint32_t kKvSmem = 6 * kTile + 1024;
 
 struct KvCtl {
-  uint64_t kv_full, q_full, s_full, p_full, mm_done, drain;
+  uint64_t kv_full, q_full[2], s_full, p_full, mm_done, drain;
   uint32_t tmem_base;
   int abort;
+  float lse2[2][kT];   // per row of a stage: forward lse in log2 units (+inf: no row)
+  float dlt[2][kT];    // D = <dout, out>
+  int tmax[2][kT];     // last key the row may attend (its token for the block's own rows)
 };
 
 // the query rows of row tile i of this key tile: the gate's groups of block j
@@ -127,6 +123,18 @@ MOBA_DEV RowTile kv_row_tile(int i, int hist_tiles, const int32_t* offsets, cons
   return rt;
 }
 
+// OR of `v` over the 256 softmax threads (named barrier 1); also a barrier
+MOBA_DEV bool softmax_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, 256, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
 __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
@@ -151,7 +159,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     mbar_init(bar(&ctl.kv_full), kSoftmaxWarps);
-    mbar_init(bar(&ctl.q_full), kSoftmaxWarps);
+    mbar_init(bar(&ctl.q_full[0]), kSoftmaxWarps);
+    mbar_init(bar(&ctl.q_full[1]), kSoftmaxWarps);
     mbar_init(bar(&ctl.s_full), 1);
     mbar_init(bar(&ctl.p_full), kSoftmaxWarps);
     mbar_init(bar(&ctl.mm_done), 1);
@@ -171,83 +180,132 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
 
   if (warp < kSoftmaxWarps) {
     const int qd = warp & 3, hf = warp >> 2;
-    const int rho = qd * 32 + lane;           // TMEM lane: a row of S/dP, a key of dK/dV
+    const int rho = qd * 32 + lane;           // TMEM lane: a key of S^T, dP^T, dK, dV
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const float sl2 = dm.scale_log2;
+    const int u = key0 + rho;                  // this thread's key
+    const bool key_ok = u < key_end;
     {
-      const int u = key0 + rho;
-      const bool ok = u < key_end;
-      const size_t kr = ((size_t)b * dm.N + (ok ? u : 0)) * dm.hkv + g;
-      load_half_row(base + kKvOffK, rho, hf, k + kr * kD, ok);
-      load_half_row(base + kKvOffV, rho, hf, v + kr * kD, ok);
+      const size_t kr = ((size_t)b * dm.N + (key_ok ? u : 0)) * dm.hkv + g;
+      load_half_row(base + kKvOffK, rho, hf, k + kr * kD, key_ok);
+      load_half_row(base + kKvOffV, rho, hf, v + kr * kD, key_ok);
       cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(&ctl.kv_full));
     }
-    bool ok = true;
-    for (int i = 0; i < ntiles && ok; ++i) {
-      if (i > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.mm_done), (i - 1) & 1, abort_flag));
-        if (!ok) break;
-      }
-      const RowTile rt = kv_row_tile(i, hist_tiles, offsets, dm, b, g, j, key0);
-      int r = 0, t = 0, h = 0;
+    // the metadata of row tile i for this thread's row (its gathered row id,
+    // lse, D and causal limit) is read one tile ahead, so a tile's copies can
+    // start as soon as its stage is free
+    struct Meta {
+      int r, tmax;
+      float lse2, dlt;
       bool valid;
+    };
+    auto meta_of = [&](int i) -> Meta {
+      Meta m{0, 0x7fffffff, INFINITY, 0.f, false};
+      if (i >= ntiles) return m;
+      const RowTile rt = kv_row_tile(i, hist_tiles, offsets, dm, b, g, j, key0);
+      int t, h;
       if (rt.own) {
         t = rt.t0 + rho;
         h = rt.h;
-        valid = t < key_end;
-        r = (b * dm.N + t) * dm.hq + h;
+        m.valid = t < key_end;
+        m.r = (b * dm.N + t) * dm.hq + h;
+        m.tmax = t;
       } else {
-        valid = rho < rt.cnt;
-        r = valid ? rows[rt.r0 + rho] : 0;
-        h = r % dm.hq;
-        t = (r / dm.hq) % dm.N;
+        m.valid = rho < rt.cnt;
+        m.r = m.valid ? rows[rt.r0 + rho] : 0;
+        h = m.r % dm.hq;
+        t = (m.r / dm.hq) % dm.N;
       }
-      load_half_row(base + kKvOffQ, rho, hf, q + (size_t)(valid ? r : 0) * kD, valid);
-      load_half_row(base + kKvOffDO, rho, hf, dout + (size_t)(valid ? r : 0) * kD, valid);
-      const float L2 = valid ? lse[((size_t)b * dm.hq + h) * dm.N + t] * kLog2e : INFINITY;
-      const float Dr = valid ? delta[r] : 0.f;
+      if (m.valid) {
+        m.lse2 = lse[((size_t)b * dm.hq + h) * dm.N + t] * kLog2e;
+        m.dlt = delta[m.r];
+      } else {
+        m.r = 0;
+      }
+      return m;
+    };
+    // row tile i into stage i & 1: this thread loads half of its row's q and
+    // dout; the hf = 0 warp writes the row's scalars
+    auto load_tile = [&](int i, const Meta& m) {
+      const int x = i & 1;
+      const uint32_t sq = base + kKvOffQ + 2u * x * kTile;
+      load_half_row(sq, rho, hf, q + (size_t)m.r * kD, m.valid);
+      load_half_row(sq + kTile, rho, hf, dout + (size_t)m.r * kD, m.valid);
       cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(&ctl.q_full));
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.s_full), i & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sr[64], dr[64];
-      tmem_ld32(tb + 64u * hf + lane_off, sr);
-      tmem_ld32(tb + 64u * hf + 32 + lane_off, sr + 32);
-      tmem_ld32(tb + 128u + 64u * hf + lane_off, dr);
-      tmem_ld32(tb + 128u + 64u * hf + 32 + lane_off, dr + 32);
-      tmem_wait_ld();
-      // keys of this warp's half valid for the row: u < key_end, and u <= t in the own block
-      const int ulim = min(key_end, rt.own ? t + 1 : key_end) - (key0 + 64 * hf);   // keys [0, ulim)
-      uint32_t pp[32], ps[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        float p0 = exp2f(__uint_as_float(sr[2 * c]) * sl2 - L2);
-        float p1 = exp2f(__uint_as_float(sr[2 * c + 1]) * sl2 - L2);
-        p0 = 2 * c < ulim ? p0 : 0.f;
-        p1 = 2 * c + 1 < ulim ? p1 : 0.f;
-        pp[c] = pack_bf16x2(p0, p1);
-        ps[c] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * c]) - Dr), p1 * (__uint_as_float(dr[2 * c + 1]) - Dr));
+      if (hf == 0) {
+        ctl.lse2[x][rho] = m.lse2;
+        ctl.dlt[x][rho] = m.dlt;
+        ctl.tmax[x][rho] = m.tmax;
       }
-      store_pairs(base + kKvOffP, rho, hf, pp);
-      store_pairs(base + kKvOffDS, rho, hf, ps);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(&ctl.p_full));
+    };
+    load_tile(0, meta_of(0));
+    Meta next = meta_of(1);
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    bool fail = softmax_any(false);   // scalars of stage 0 visible to every softmax thread
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(bar(&ctl.kv_full));
+      mbar_arrive(bar(&ctl.q_full[0]));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.mm_done), (ntiles - 1) & 1, abort_flag));
-    if (ok) {
+    for (int i = 0; i < ntiles; ++i) {
+      const int x = i & 1;
+      const bool more = i + 1 < ntiles;
+      if (more) {
+        // stage x ^ 1 held row tile i - 1: free once its MMAs completed
+        if (i >= 1 && !fail)
+          fail = !__all_sync(0xffffffffu, mbar_wait(bar(&ctl.mm_done), (i - 1) & 1, abort_flag));
+        if (!fail) {
+          load_tile(i + 1, next);
+          next = meta_of(i + 2);
+        }
+      }
+      if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(bar(&ctl.s_full), i & 1, abort_flag));
+      if (!fail) {
+        tc_fence_after();
+        uint32_t sr[64], dr[64];
+        tmem_ld32(tb + 64u * hf + lane_off, sr);
+        tmem_ld32(tb + 64u * hf + 32 + lane_off, sr + 32);
+        tmem_ld32(tb + 128u + 64u * hf + lane_off, dr);
+        tmem_ld32(tb + 128u + 64u * hf + 32 + lane_off, dr + 32);
+        tmem_wait_ld();
+        uint32_t pp[32], ps[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int ra = 64 * hf + 2 * c, rb = ra + 1;   // rows of this column pair
+          float p0 = ex2_approx(__uint_as_float(sr[2 * c]) * sl2 - ctl.lse2[x][ra]);
+          float p1 = ex2_approx(__uint_as_float(sr[2 * c + 1]) * sl2 - ctl.lse2[x][rb]);
+          p0 = (key_ok && u <= ctl.tmax[x][ra]) ? p0 : 0.f;
+          p1 = (key_ok && u <= ctl.tmax[x][rb]) ? p1 : 0.f;
+          pp[c] = pack_bf16x2(p0, p1);
+          ps[c] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * c]) - ctl.dlt[x][ra]),
+                              p1 * (__uint_as_float(dr[2 * c + 1]) - ctl.dlt[x][rb]));
+        }
+        // P^T and dS^T over this warp's own S^T / dP^T columns [64 hf, 64 hf + 32): already read
+        tmem_st32(tb + 64u * hf + lane_off, pp);
+        tmem_st32(tb + 128u + 64u * hf + lane_off, ps);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(&ctl.p_full));
+      }
+      if (more) {
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+      }
+      // one barrier per tile: the next stage's scalars are visible, and every
+      // softmax warp learns of a failure in any of them
+      if (softmax_any(fail)) {
+        fail = true;
+        break;
+      }
+      __syncwarp();
+      if (more && lane == 0) mbar_arrive(bar(&ctl.q_full[x ^ 1]));
+    }
+    if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(bar(&ctl.mm_done), (ntiles - 1) & 1, abort_flag));
+    if (!fail) {
       // dK, dV rows (lanes = keys) of this warp's 64 columns
       tc_fence_after();
-      const int u = key0 + rho;
       const float scale = sl2 / kLog2e;
       const size_t kr = ((size_t)b * dm.N + u) * dm.hkv + g;
 #pragma unroll
@@ -256,7 +314,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
         tmem_ld32(tb + 256u + 64u * hf + 32u * cc + lane_off, gvv);
         tmem_ld32(tb + 384u + 64u * hf + 32u * cc + lane_off, gkk);
         tmem_wait_ld();
-        if (u < key_end) {
+        if (key_ok) {
           uint4* dvp = reinterpret_cast<uint4*>(dv + kr * kD + 64 * hf + 32 * cc);
           uint4* dkp = reinterpret_cast<uint4*>(dk + kr * kD + 64 * hf + 32 * cc);
 #pragma unroll
@@ -277,40 +335,43 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
     }
   } else if (lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t idS = idesc_bf16(128, kT, false);          // A, B K-major
-    const uint32_t idG = idesc_bf16_amn(128, kD, true);       // A, B MN-major
+    const uint32_t idS = idesc_bf16(128, kT, false);     // A, B K-major
+    const uint32_t idG = idesc_bf16(128, kD, true);      // A from TMEM, B MN-major
     const uint32_t hi = sdesc_hi(1024);
-    const uint32_t loK = sdesc_lo(base + kKvOffK, 16), loV = sdesc_lo(base + kKvOffV, 16),
-                   loQ = sdesc_lo(base + kKvOffQ, 16), loDO = sdesc_lo(base + kKvOffDO, 16);
-    const uint32_t mnQ = sdesc_lo(base + kKvOffQ, kHalf), mnDO = sdesc_lo(base + kKvOffDO, kHalf),
-                   mnP = sdesc_lo(base + kKvOffP, kHalf), mnDS = sdesc_lo(base + kKvOffDS, kHalf);
+    const uint32_t loK = sdesc_lo(base + kKvOffK, 16), loV = sdesc_lo(base + kKvOffV, 16);
     bool ok = mbar_wait(bar(&ctl.kv_full), 0, abort_flag);
     for (int i = 0; i < ntiles && ok; ++i) {
-      if (!(ok = mbar_wait(bar(&ctl.q_full), i & 1, abort_flag))) break;
+      const int x = i & 1;
+      const uint32_t sq = base + kKvOffQ + 2u * x * kTile, sdo = sq + kTile;
+      const uint32_t loQ = sdesc_lo(sq, 16), loDO = sdesc_lo(sdo, 16);
+      const uint32_t mnQ = sdesc_lo(sq, kHalf), mnDO = sdesc_lo(sdo, kHalf);
+      if (!(ok = mbar_wait(bar(&ctl.q_full[x]), (i >> 1) & 1, abort_flag))) break;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-        mma_ss(tb, sdesc_join(loQ + off, hi), sdesc_join(loK + off, hi), idS, kk > 0);
+        mma_ss(tb, sdesc_join(loK + off, hi), sdesc_join(loQ + off, hi), idS, kk > 0);
       }
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-        mma_ss(tb + 128u, sdesc_join(loDO + off, hi), sdesc_join(loV + off, hi), idS, kk > 0);
+        mma_ss(tb + 128u, sdesc_join(loV + off, hi), sdesc_join(loDO + off, hi), idS, kk > 0);
       }
       mma_commit(bar(&ctl.s_full));
       if (!(ok = mbar_wait(bar(&ctl.p_full), i & 1, abort_flag))) break;
       tc_fence_after();
-      // dV += P^T dO and dK += dS^T Q: K runs over the 128 rows, 16 per MMA
+      // dV += P^T dO, dK += dS^T Q: K runs over the 128 rows (rows 0-63 in
+      // columns 0-31 of P^T / dS^T, rows 64-127 in columns 64-95)
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk * 2048) >> 4;
-        mma_ss(tb + 256u, sdesc_join(mnP + off, hi), sdesc_join(mnDO + off, hi), idG, (i > 0 || kk > 0) ? 1u : 0u);
+        const uint32_t a = kk < 4 ? kk * 8u : 64u + (kk - 4) * 8u;
+        mma_ts(tb + 256u, tb + a, sdesc_join(mnDO + ((kk * 2048) >> 4), hi), idG, (i > 0 || kk > 0) ? 1u : 0u);
       }
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk * 2048) >> 4;
-        mma_ss(tb + 384u, sdesc_join(mnDS + off, hi), sdesc_join(mnQ + off, hi), idG, (i > 0 || kk > 0) ? 1u : 0u);
+        const uint32_t a = kk < 4 ? kk * 8u : 64u + (kk - 4) * 8u;
+        mma_ts(tb + 384u, tb + 128u + a, sdesc_join(mnQ + ((kk * 2048) >> 4), hi), idG,
+               (i > 0 || kk > 0) ? 1u : 0u);
       }
       mma_commit(bar(&ctl.mm_done));
     }
@@ -456,8 +517,8 @@ __global__ void __launch_bounds__(kQThreads, 1) bwd_q_tc_kernel(
       uint32_t ps[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        float p0 = exp2f(__uint_as_float(sr[2 * c]) * sl2 - L2);
-        float p1 = exp2f(__uint_as_float(sr[2 * c + 1]) * sl2 - L2);
+        float p0 = ex2_approx(__uint_as_float(sr[2 * c]) * sl2 - L2);
+        float p1 = ex2_approx(__uint_as_float(sr[2 * c + 1]) * sl2 - L2);
         p0 = (2 * c >= vlo && 2 * c <= vhi) ? p0 : 0.f;
         p1 = (2 * c + 1 >= vlo && 2 * c + 1 <= vhi) ? p1 : 0.f;
         ps[c] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * c]) - Dr), p1 * (__uint_as_float(dr[2 * c + 1]) - Dr));
