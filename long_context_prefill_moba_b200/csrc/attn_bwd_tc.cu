@@ -69,8 +69,12 @@ constexpr int kKvThreads = (kSoftmaxWarps + 1) * 32;
 constexpr uint32_t kKvOffK = 0, kKvOffV = kTile, kKvOffQ = 2 * kTile;   // Q/dO stage x at kKvOffQ + 2x kTile
 constexpr uint32_t kKvSmem = 6 * kTile + 1024;
 
+constexpr int kMaxPassPrefix = 256;    // passes whose row-tile prefix is kept in shared memory
+
 struct KvCtl {
   uint64_t kv_full, q_full[2], s_full, p_full, mm_done, drain;
+  int pass_tiles[kMaxPassPrefix + 1];   // routed row tiles of passes [0, p), this CTA's group
+  int pass_r0[kMaxPassPrefix];          // first routed row of pass p's group
   uint32_t tmem_base;
   int abort;
   float lse2[2][kT];   // per row of a stage: forward lse in log2 units (+inf: no row)
@@ -98,8 +102,23 @@ MOBA_DEV int kv_tiles(const int32_t* offsets, const Dims& dm, int b, int g, int 
 }
 
 MOBA_DEV RowTile kv_row_tile(int i, int hist_tiles, const int32_t* offsets, const Dims& dm, int b, int g, int j,
-                             int key0) {
+                             int key0, const int* pass_tiles, const int* pass_r0) {
   RowTile rt{};
+  if (i < hist_tiles && pass_tiles != nullptr) {
+    // the pass holding tile i: largest p with pass_tiles[p] <= i
+    int lo = 0, hi = dm.nchunks - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pass_tiles[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    const int left = i - pass_tiles[lo];
+    const int64_t ngroups = (int64_t)dm.batch * dm.hkv * dm.n;
+    const int64_t gi = lo * ngroups + ((int64_t)b * dm.hkv + g) * dm.n + j;
+    rt.own = false;
+    rt.r0 = pass_r0[lo] + left * kT;
+    rt.cnt = min(kT, offsets[gi + 1] - rt.r0);
+    return rt;
+  }
   if (i < hist_tiles) {
     const int64_t ngroups = (int64_t)dm.batch * dm.hkv * dm.n;
     int left = i;
@@ -157,6 +176,20 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
   const int ntiles = kv_tiles(offsets, dm, b, g, j, key0, key_end, hist_tiles);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool prefix = dm.nchunks <= kMaxPassPrefix;
+  if (prefix && tid == 0) {
+    const int64_t ngroups = (int64_t)dm.batch * dm.hkv * dm.n;
+    int acc = 0;
+    for (int ch = 0; ch < dm.nchunks; ++ch) {
+      const int64_t gi = ch * ngroups + ((int64_t)b * dm.hkv + g) * dm.n + j;
+      ctl.pass_tiles[ch] = acc;
+      ctl.pass_r0[ch] = offsets[gi];
+      acc += (offsets[gi + 1] - offsets[gi] + kT - 1) / kT;
+    }
+    ctl.pass_tiles[dm.nchunks] = acc;
+  }
+  const int* pt = prefix ? ctl.pass_tiles : nullptr;
+  const int* pr = prefix ? ctl.pass_r0 : nullptr;
   if (tid == 0) {
     mbar_init(bar(&ctl.kv_full), kSoftmaxWarps);
     mbar_init(bar(&ctl.q_full[0]), kSoftmaxWarps);
@@ -202,7 +235,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
     auto meta_of = [&](int i) -> Meta {
       Meta m{0, 0x7fffffff, INFINITY, 0.f, false};
       if (i >= ntiles) return m;
-      const RowTile rt = kv_row_tile(i, hist_tiles, offsets, dm, b, g, j, key0);
+      const RowTile rt = kv_row_tile(i, hist_tiles, offsets, dm, b, g, j, key0, pt, pr);
       int t, h;
       if (rt.own) {
         t = rt.t0 + rho;
