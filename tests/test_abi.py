@@ -104,6 +104,44 @@ def test_entry_points_validate_before_launching(L):
     assert L.moba_last_launch_count() == 0
 
 
+def test_backward_and_host_entry_points_validate_before_launching(L):
+    s = shape(seqlen=4096, block=256)
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    P = ctypes.byref(s)
+    big = 1 << 40
+    # moba_attn_bwd(shape, q, k, v, out, dout, lse, sel, offsets, rows, dq, dk, dv, ws, ws_bytes, stream)
+    args = [fake] * 13
+    assert L.moba_attn_bwd(P, *args[:12], fake, 16, None) == 3                  # workspace too small
+    nul = list(args)
+    nul[4] = None                                                                # dout missing
+    assert L.moba_attn_bwd(P, *nul[:12], fake, big, None) == 1
+    mis = list(args)
+    mis[9] = odd                                                                 # dq misaligned
+    assert L.moba_attn_bwd(P, *mis[:12], fake, big, None) == 1
+    bad = shape(hq=5, hkv=2)
+    assert L.moba_attn_bwd(ctypes.byref(bad), *args[:12], fake, big, None) == 1
+    # moba_prefill_host(shape, q, k, v, out, lse, status, ws, ws_bytes, stream)
+    assert L.moba_prefill_host(P, fake, fake, fake, fake, None, None, fake, 16, None) == 3
+    assert L.moba_prefill_host(P, None, fake, fake, fake, None, None, fake, big, None) == 1
+    assert L.moba_prefill_host(P, fake, fake, fake, fake, None, None, odd, big, None) == 1
+    assert L.moba_last_launch_count() == 0
+
+
+def test_backward_and_host_workspace_sizes(L):
+    s = shape()                                   # the 1M bf16 layer: tensor-core backward
+    n_q = (1 << 20) * 32 * 128
+    n_k = (1 << 20) * 8 * 128
+    assert M.moba_attn_bwd_workspace_size(s) >= n_q * 4 + (1 << 20) * 32 * 4   # dq accumulator + delta
+    f = shape(seqlen=4096, block=256, dtype="f32", head_dim=64)
+    assert 0 < M.moba_attn_bwd_workspace_size(f) < 4096 * 32 * 64 * 4      # no dq accumulator
+    no_lse = M.moba_prefill_host_workspace_size(s, False)
+    with_lse = M.moba_prefill_host_workspace_size(s, True)
+    assert no_lse >= 2 * (n_q + n_k) * 2 + M.moba_attn_workspace_size(s) + M.moba_gate_workspace_size(s)
+    assert with_lse - no_lse >= (1 << 20) * 32 * 4 - 256      # an empty region still takes 256 B
+    assert M.moba_prefill_host_workspace_size(shape(hq=5, hkv=2), False) == 0
+
+
 def test_status_strings(L):
     for st in range(7):
         assert M.moba_status_string(st).startswith("MOBA_")
