@@ -233,16 +233,17 @@ MOBA_API size_t moba_prefill_host_workspace_size(const moba_shape_t* shape, int 
  *   ws       >= moba_prefill_host_workspace_size(shape, lse != NULL) bytes of
  *            device memory, 16-byte aligned; it holds the device copies of the
  *            tensors and every intermediate array
- * k and v are copied in first (mean-pool starts when they land); q arrives one
- * query pass (moba_query_chunk tokens) at a time on a second stream, the gate
- * and the attention of a pass start as soon as its queries are in, and each
- * pass's output returns on a third stream while the next pass computes.  The
- * call only enqueues: `stream` (the compute stream) completes when the last
- * output byte is in host memory.  The copies overlap only from page-locked
- * host memory (cudaHostAlloc / cudaHostRegister); pageable buffers give the
- * same results with copies that block the calling thread.  The call creates
- * and releases two streams and 2 * (passes + 2) events; it does no device
- * allocation. */
+ * q, k and v arrive one query pass (moba_query_chunk tokens) at a time on a
+ * second stream (every step of a pass reads only tokens before the pass's
+ * end); the mean-pool of the blocks a pass completes, its gate and its
+ * attention start as soon as its rows are in, and each pass's output returns
+ * on a third stream while the next pass computes.  The device copies of k and
+ * v are cleared first.  The call only enqueues: `stream` (the compute stream)
+ * completes when the last output byte is in host memory.  The copies overlap
+ * only from page-locked host memory (cudaHostAlloc / cudaHostRegister);
+ * pageable buffers give the same results with copies that block the calling
+ * thread.  The call creates and releases two streams and 2 * passes + 2
+ * events; it does no device allocation. */
 MOBA_API moba_status_t moba_prefill_host(const moba_shape_t* shape, const void* q, const void* k,
                                          const void* v, void* out, float* lse, int* status,
                                          void* ws, size_t ws_bytes, moba_stream_t stream);

@@ -17,6 +17,9 @@ int64_t hist_rows_range(int64_t t0, int64_t t1, int64_t B, int64_t KH);
 
 cudaError_t launch_meanpool(const Dims& dm, int dtype, const void* k, float* meank,
                             cudaStream_t stream, int* launches);
+// blocks [j0, j1) only
+cudaError_t launch_meanpool_blocks(const Dims& dm, int dtype, const void* k, float* meank, int j0,
+                                   int j1, cudaStream_t stream, int* launches);
 
 struct GateWs {
   int32_t* counts;   // [ngroups] rows per (chunk, b, g, j)

@@ -20,7 +20,7 @@ constexpr int kUnroll = 4;
 template <typename T>
 __global__ void __launch_bounds__(kThreads) meanpool_kernel(const T* __restrict__ k,
                                                             float* __restrict__ meank, int N, int W,
-                                                            int B, int n) {
+                                                            int B, int n, int j0) {
   constexpr int V = Vec16<T>::kN;            // elements per 16-byte load
   const int vecs_per_row = W / V;             // W = hkv * d is a multiple of V
   const int cols_cta = min(vecs_per_row, kThreads);
@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(kThreads) meanpool_kernel(const T* __restrict_
   const int tid = threadIdx.x;
   const int cvec = blockIdx.x * cols_cta + (tid % cols_cta);
   const int rsub = tid / cols_cta;
-  const int j = blockIdx.y;
+  const int j = j0 + blockIdx.y;
   const int b = blockIdx.z;
   const int t0 = j * B;
   const int t1 = min(N, t0 + B);
@@ -77,21 +77,27 @@ __global__ void __launch_bounds__(kThreads) meanpool_kernel(const T* __restrict_
 
 }  // namespace
 
-cudaError_t launch_meanpool(const Dims& dm, int dtype, const void* k, float* meank,
-                            cudaStream_t stream, int* launches) {
+cudaError_t launch_meanpool_blocks(const Dims& dm, int dtype, const void* k, float* meank, int j0,
+                                   int j1, cudaStream_t stream, int* launches) {
+  if (j1 <= j0) return cudaSuccess;
   const int W = dm.hkv * dm.d;
   const int V = dtype == MOBA_BF16 ? 8 : 4;
   const int vecs_per_row = W / V;
   const int cols_cta = vecs_per_row < kThreads ? vecs_per_row : kThreads;
-  dim3 grid((vecs_per_row + cols_cta - 1) / cols_cta, dm.n, dm.batch);
+  dim3 grid((vecs_per_row + cols_cta - 1) / cols_cta, j1 - j0, dm.batch);
   if (dtype == MOBA_BF16)
     meanpool_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(k), meank, dm.N, W, dm.B, dm.n);
+        static_cast<const __nv_bfloat16*>(k), meank, dm.N, W, dm.B, dm.n, j0);
   else
     meanpool_kernel<float><<<grid, kThreads, 0, stream>>>(static_cast<const float*>(k), meank, dm.N,
-                                                           W, dm.B, dm.n);
+                                                           W, dm.B, dm.n, j0);
   ++*launches;
   return cudaGetLastError();
+}
+
+cudaError_t launch_meanpool(const Dims& dm, int dtype, const void* k, float* meank,
+                            cudaStream_t stream, int* launches) {
+  return launch_meanpool_blocks(dm, dtype, k, meank, 0, dm.n, stream, launches);
 }
 
 }  // namespace moba

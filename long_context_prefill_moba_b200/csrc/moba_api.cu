@@ -346,44 +346,61 @@ MOBA_API moba_status_t moba_prefill_host(const moba_shape_t* s, const void* q, c
   // object made here is released at the end (destroying a stream or event
   // with work pending is legal: it goes once that work is done)
   cudaStream_t s_in = nullptr, s_out = nullptr;
-  cudaEvent_t ev_start = nullptr, ev_kv = nullptr, ev_done = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_done = nullptr;
   cudaEvent_t* ev_q = new cudaEvent_t[np]();
   cudaEvent_t* ev_o = new cudaEvent_t[np]();
   int launches = 0;
   cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
-  for (cudaEvent_t* ev : {&ev_start, &ev_kv, &ev_done})
+  for (cudaEvent_t* ev : {&ev_start, &ev_done})
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
   for (int p = 0; p < np && e == cudaSuccess; ++p) {
     e = cudaEventCreateWithFlags(&ev_q[p], cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_o[p], cudaEventDisableTiming);
   }
+  // k and v stream in with the passes, so a tile that reaches past the copied
+  // rows (masked, but multiplied by zero probabilities) must read finite
+  // values: clear the device copies first
+  if (e == cudaSuccess) e = cudaMemsetAsync(kd, 0, kbytes, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(vd, 0, kbytes, stream);
   // the copies start after the work already queued on the caller's stream
   if (e == cudaSuccess) e = cudaEventRecord(ev_start, stream);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_start, 0);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_start, 0);
-  // host -> device: k and v whole, then q one query pass at a time
-  if (e == cudaSuccess) e = cudaMemcpyAsync(kd, k, kbytes, cudaMemcpyHostToDevice, s_in);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(vd, v, kbytes, cudaMemcpyHostToDevice, s_in);
-  if (e == cudaSuccess) e = cudaEventRecord(ev_kv, s_in);
+  // host -> device one query pass at a time: the pass's k, v and q rows.  Every
+  // step of pass p reads only tokens before the pass's end: the pooled keys of
+  // complete blocks, the gate's candidate blocks (all earlier) and the
+  // attention's keys.
+  const size_t krow = (size_t)s->hkv * s->head_dim * es;
   for (int p = 0; p < np && e == cudaSuccess; ++p) {
     const int t0 = p * dm.chunk, t1 = dm.N < t0 + dm.chunk ? dm.N : t0 + dm.chunk;
+    const size_t kp = (size_t)dm.N * krow;
+    e = cudaMemcpy2DAsync(static_cast<char*>(kd) + (size_t)t0 * krow, kp, static_cast<const char*>(k) + (size_t)t0 * krow,
+                          kp, (size_t)(t1 - t0) * krow, dm.batch, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(static_cast<char*>(vd) + (size_t)t0 * krow, kp,
+                            static_cast<const char*>(v) + (size_t)t0 * krow, kp, (size_t)(t1 - t0) * krow,
+                            dm.batch, cudaMemcpyHostToDevice, s_in);
     const size_t pitch = (size_t)dm.N * qrow;
-    e = cudaMemcpy2DAsync(static_cast<char*>(qd) + (size_t)t0 * qrow, pitch,
-                          static_cast<const char*>(q) + (size_t)t0 * qrow, pitch, (size_t)(t1 - t0) * qrow,
-                          dm.batch, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(static_cast<char*>(qd) + (size_t)t0 * qrow, pitch,
+                            static_cast<const char*>(q) + (size_t)t0 * qrow, pitch, (size_t)(t1 - t0) * qrow,
+                            dm.batch, cudaMemcpyHostToDevice, s_in);
     if (e == cudaSuccess) e = cudaEventRecord(ev_q[p], s_in);
   }
-  // compute on the caller's stream: mean-pool once k is in, then gate and
-  // attention pass by pass as each pass's queries arrive
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, ev_kv, 0);
-  if (e == cudaSuccess) e = moba::launch_meanpool(dm, s->dtype, kd, meank, stream, &launches);
+  // compute on the caller's stream, pass by pass as each pass's rows arrive:
+  // mean-pool of the blocks the pass completes, gate, attention
   if (e == cudaSuccess) e = cudaMemsetAsync(g.counts, 0, sizeof(int32_t) * G * 2, stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(g.status, 0, sizeof(int), stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(a.status, 0, sizeof(int), stream);
+  int pooled = 0;
   for (int p = 0; p < np && e == cudaSuccess; ++p) {
     const int t0 = p * dm.chunk, t1 = dm.N < t0 + dm.chunk ? dm.N : t0 + dm.chunk;
     e = cudaStreamWaitEvent(stream, ev_q[p], 0);
+    const int upto = t1 == dm.N ? dm.n : t1 / dm.B;   // blocks complete once the pass is in
+    if (e == cudaSuccess)
+      e = moba::launch_meanpool_blocks(dm, s->dtype, kd, meank, pooled, upto, stream, &launches);
+    pooled = upto > pooled ? upto : pooled;
     if (e == cudaSuccess)
       e = moba::launch_gate_pass(dm, s->dtype, qd, meank, sel, offsets, rows, g, p, stream, &launches);
     if (e == cudaSuccess)
@@ -416,7 +433,7 @@ MOBA_API moba_status_t moba_prefill_host(const moba_shape_t* s, const void* q, c
   }
   delete[] ev_q;
   delete[] ev_o;
-  for (cudaEvent_t ev : {ev_start, ev_kv, ev_done})
+  for (cudaEvent_t ev : {ev_start, ev_done})
     if (ev != nullptr) cudaEventDestroy(ev);
   if (s_in != nullptr) cudaStreamDestroy(s_in);
   if (s_out != nullptr) cudaStreamDestroy(s_out);
