@@ -27,6 +27,10 @@ CASES = {
     # tensor-core path with several row tiles per key tile and four passes
     "bf16_multitile": (S.get_config("mqar").replace(batch=1, seqlen=4096, hq=8, hkv=2, block=512, topk=4),
                        1024),
+    # eight query heads on one kv head (GQA 8) on tensor cores
+    "gqa8_bf16": (S.get_config("mqar").replace(batch=1, seqlen=1024, hq=8, hkv=1, block=64, topk=5), 384),
+    # one-token blocks: every key tile straddles many blocks
+    "block_one": (S.get_config("mqar").replace(batch=1, seqlen=200, hq=2, hkv=1, block=1, topk=3), 0),
 }
 
 
@@ -62,6 +66,26 @@ def test_backward_parity(cuda_device, name):
         err = float(np.abs(cpu(got).numpy() - ref).max())
         print(name, name_, "max abs err", err, "max |ref|", float(np.abs(ref).max()))
         assert err <= tol(cfg, ref), (name_, err)
+
+
+def test_dense_special_case_backward_matches_autograd(cuda_device):
+    # top-k >= n: MoBA is dense causal attention, so its gradients are those of
+    # torch's causal SDPA (autograd in fp32 on the same bf16 inputs)
+    cfg = S.get_config("mqar").replace(batch=1, seqlen=640, hq=4, hkv=2, block=64, topk=16)
+    res, dq, dk, dv = run_backward(cfg, 0)
+    rep = cfg.hq // cfg.hkv
+    q = res["q"].float().transpose(1, 2).detach().requires_grad_(True)
+    k = res["k"].float().detach().requires_grad_(True)
+    v = res["v"].float().detach().requires_grad_(True)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        q, k.repeat_interleave(rep, 2).transpose(1, 2), v.repeat_interleave(rep, 2).transpose(1, 2),
+        is_causal=True, scale=cfg.softmax_scale)
+    dout = S.gen_dout(cfg, res["q"].device).float().transpose(1, 2)
+    (out * dout).sum().backward()
+    for name_, got, ref in (("dq", dq.float(), q.grad.transpose(1, 2)), ("dk", dk.float(), k.grad),
+                            ("dv", dv.float(), v.grad)):
+        err = (got - ref).abs().max().item()
+        assert err <= 3e-2 * max(1.0, ref.abs().max().item()), (name_, err)
 
 
 @pytest.mark.parametrize("name", ["ragged_multipass", "d64_bf16"])
