@@ -71,10 +71,13 @@ struct AttnLayout {
 AttnLayout attn_layout(const moba_shape_t* s) {
   const size_t KH = s->topk - 1;
   const size_t entries = (size_t)s->batch * chunk_of(s) * s->hq * KH;
+  // the tensor-core kernels (bf16, head_dim 128) keep the partial outputs in
+  // bf16; the others in fp32
+  const size_t part_bytes = s->dtype == MOBA_BF16 && s->head_dim == 128 ? 2 : 4;
   AttnLayout L;
   L.status = 0;
   L.part_o = 256;
-  L.part_lse = L.part_o + align_up(entries * s->head_dim * sizeof(float));
+  L.part_lse = L.part_o + align_up(entries * s->head_dim * part_bytes);
   L.tile_start = L.part_lse + align_up(entries * sizeof(float));
   L.total = L.tile_start + align_up(((size_t)s->batch * s->hkv * nblocks(s) + 1) * sizeof(int32_t));
   return L;
