@@ -243,7 +243,8 @@ MOBA_API size_t moba_prefill_host_workspace_size(const moba_shape_t* shape, int 
  * only from page-locked host memory (cudaHostAlloc / cudaHostRegister);
  * pageable buffers give the same results with copies that block the calling
  * thread.  The call creates and releases two streams and 2 * passes + 2
- * events; it does no device allocation. */
+ * events; it does no device allocation.  If a CUDA call fails after copies
+ * were queued, it waits for them before returning MOBA_ERR_CUDA. */
 MOBA_API moba_status_t moba_prefill_host(const moba_shape_t* shape, const void* q, const void* k,
                                          const void* v, void* out, float* lse, int* status,
                                          void* ws, size_t ws_bytes, moba_stream_t stream);

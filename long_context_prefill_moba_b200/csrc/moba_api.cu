@@ -430,6 +430,12 @@ MOBA_API moba_status_t moba_prefill_host(const moba_shape_t* s, const void* q, c
   // the caller's stream completes only after the last copy-out
   if (e == cudaSuccess) e = cudaEventRecord(ev_done, s_out);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, ev_done, 0);
+  if (e != cudaSuccess) {
+    // the caller's stream may not cover copies already queued on the private
+    // streams: let them finish before the caller can release its buffers
+    if (s_in != nullptr) cudaStreamSynchronize(s_in);
+    if (s_out != nullptr) cudaStreamSynchronize(s_out);
+  }
   for (int p = 0; p < np; ++p) {
     if (ev_q[p] != nullptr) cudaEventDestroy(ev_q[p]);
     if (ev_o[p] != nullptr) cudaEventDestroy(ev_o[p]);
