@@ -72,10 +72,6 @@ MOBA_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, ui
 MOBA_DEV void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
-// cp.async completions of this thread arrive on the mbarrier (no pending count increment)
-MOBA_DEV void cp_async_mbar_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
-}
 
 // ---- tcgen05: TMEM allocation ------------------------------------------------
 MOBA_DEV void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {   // whole warp
@@ -120,10 +116,6 @@ MOBA_DEV void mma_commit(uint32_t bar) {
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-// the same with the A operand read MN-major from shared memory (bit 15)
-__host__ __device__ constexpr uint32_t idesc_bf16_amn(int M, int N, bool b_mn_major) {
-  return idesc_bf16(M, N, b_mn_major) | (1u << 15);
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle:
@@ -174,14 +166,6 @@ MOBA_DEV void tmem_st32(uint32_t taddr, const uint32_t* r) {
       "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
-MOBA_DEV void tmem_st16(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15,%16};\n" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
 MOBA_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 MOBA_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
@@ -225,24 +209,14 @@ MOBA_DEV float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe (offloads the special-function unit in the softmax).
-// x = n + f with n = rint(x) (by the 1.5 * 2^23 rounding trick) and
-// f in [-0.5, 0.5]; 2^f is a degree-3 polynomial fitted in this project by
-// iteratively reweighted least squares on the relative error (max relative
-// error 7.5e-5, far below the 2^-9 rounding of the bf16 probabilities it
-// feeds); 2^n is added to the exponent field.  Inputs below -126 give ~1e-38.
-MOBA_DEV float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float r = x + 12582912.f;
-  const float f = x - (r - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.05517206f, f, 0.24261241f), f, 0.69326101f), f, 0.99992796f);
-  const int n = __float_as_int(r) - 0x4B400000;   // bits of 12582912.f
-  return __int_as_float(__float_as_int(p) + (n << 23));
-}
-
-// exp2_poly on a packed pair: the same clamp, range reduction, polynomial and
-// exponent insertion, bit for bit, with the fp32 steps as paired instructions
-// (three adds/subtracts and three FMAs per pair on the FMA pipe).
+// 2^x for a packed pair of fp32 values on the FMA pipe (an alternative to the
+// special-function unit in the softmax).  x is clamped at -126, x = n + f with
+// n = rint(x) (by the 1.5 * 2^23 rounding trick) and f in [-0.5, 0.5]; 2^f is a
+// degree-3 polynomial fitted in this project by iteratively reweighted least
+// squares on the relative error (max relative error 7.5e-5, far below the 2^-9
+// rounding of the bf16 probabilities it feeds); 2^n is added to the exponent
+// field.  Inputs below -126 give ~1e-38.  The fp32 steps run as paired
+// instructions (three adds/subtracts and three FMAs per pair).
 MOBA_DEV uint64_t exp2_poly2(uint64_t x2) {
   float a, b;
   f2_unpack(x2, a, b);

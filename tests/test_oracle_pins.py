@@ -308,7 +308,7 @@ def test_algorithmic_pairs_brute_force(N, B, topk):
 
 # --------------------------------------------------------------------------
 # the FMA-pipe exponential used for part of the softmax (csrc/sm100.cuh,
-# exp2_poly): its fitted polynomial's relative error bound, checked in fp32
+# exp2_poly2, per lane): its fitted polynomial's relative error bound, checked in fp32
 # arithmetic against the exact 2^x over the range the softmax uses
 # --------------------------------------------------------------------------
 def test_exp2_polynomial_error_bound():
