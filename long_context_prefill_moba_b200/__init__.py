@@ -32,7 +32,7 @@ __all__ = [
     "moba_attn_workspace_size", "moba_block_meanpool", "moba_gate_topk", "moba_attn_fwd",
     "moba_status_string", "moba_last_launch_count", "moba_gate_topk_noalloc", "MobaLayer", "moba_forward",
     "moba_prefill_host_workspace_size", "moba_prefill_host", "MobaHostLayer",
-    "moba_attn_bwd_workspace_size", "moba_attn_bwd",
+    "moba_attn_bwd_workspace_size", "moba_attn_bwd", "moba_attention",
     "MOBA_BF16", "MOBA_F32", "EXPORTED_SYMBOLS",
 ]
 
@@ -346,3 +346,33 @@ def moba_forward(q, k, v, block, topk, scale=None, return_lse=False, query_chunk
     lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device) if return_lse else None
     layer.forward(q, k, v, out, lse)
     return (out, lse) if return_lse else out
+
+
+class _MobaAttention(torch.autograd.Function):
+    """MoBA attention as a differentiable op: the forward runs the three steps,
+    the backward moba_attn_bwd with the forward's selection held fixed."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, block, topk, scale, query_chunk):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        b, N, hq, d = q.shape
+        layer = MobaLayer(b, N, hq, k.shape[2], d, block, topk, q.dtype, scale, query_chunk, q.device)
+        out = torch.empty_like(q)
+        lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device)
+        layer.forward(q, k, v, out, lse)
+        ctx.layer = layer
+        ctx.save_for_backward(q, k, v, out, lse)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse = ctx.saved_tensors
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ctx.layer.backward(q, k, v, out, lse, dout.contiguous(), dq, dk, dv)
+        return dq, dk, dv, None, None, None, None
+
+
+def moba_attention(q, k, v, block, topk, scale=None, query_chunk=0):
+    """Differentiable MoBA attention: q [b,N,Hq,d], k/v [b,N,Hkv,d] CUDA tensors
+    -> out [b,N,Hq,d]; gradients flow to q, k, v (not through the block selection)."""
+    return _MobaAttention.apply(q, k, v, block, topk, scale, query_chunk)
