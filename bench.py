@@ -394,12 +394,14 @@ def main():
         return
     cfg = S.get_config(args.config)
 
-    world, rank, local = dist_setup()
     if args.impl == "reference":
-        if rank == 0:
+        # the CPU oracle needs no process group: under torchrun rank 0 runs it and
+        # the other ranks exit at once
+        if int(os.environ.get("RANK", "0")) == 0:
             run_reference(args, cfg)
-        barrier(world)
         return
+
+    world, rank, local = dist_setup()
 
     import long_context_prefill_moba_b200 as M
     M.load_library()
