@@ -47,3 +47,16 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(12.5, 1) == 12.5
     assert bench.job_throughput(3.0, 1000.0, 1) == pytest.approx(3.0)
+
+
+def test_traffic_record_matches_the_attention_source():
+    # bench.py reports the ncu-measured DRAM traffic only while csrc/attn_tc.cu is
+    # the source it was captured from; a kernel edit must come with a new capture
+    import hashlib
+    import json
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    rec = json.load(open(os.path.join(root, "profiles", "attn_traffic.json")))
+    src = open(os.path.join(root, "long_context_prefill_moba_b200", "csrc", "attn_tc.cu"), "rb").read()
+    assert hashlib.sha256(src).hexdigest() == rec["kernel_source_sha256"]
+    assert 0 < rec["dram_bytes_per_row"] < 4096
