@@ -249,6 +249,67 @@ MOBA_API moba_status_t moba_prefill_host(const moba_shape_t* shape, const void* 
                                          const void* v, void* out, float* lse, int* status,
                                          void* ws, size_t ws_bytes, moba_stream_t stream);
 
+/* ---- gate variant: mean-, max- and min-pooled block keys ----------------- */
+
+/* [review], the authors' rebuttals to W1 (block representation; the comparison
+ * with QUEST): an ablation that, besides the blocks the mean-pooled gate
+ * selects, also selects the top blocks under max pooling and under min pooling
+ * of the keys.  The page gives no formula.  The reading implemented here: a
+ * query at position t (current block c) attends
+ *     the top (topk - 1) earlier blocks by <q, mean K_j>   (the plain gate)
+ *   U the top `extra` earlier blocks by <q, max K_j>
+ *   U the top `extra` earlier blocks by <q, min K_j>
+ *   U {c},
+ * max and min taken channel-wise over the block's key rows, each ranking over
+ * the blocks j < c with equal scores going to the lower block index.  With
+ * extra = 0 this is the plain gate.  A row attends between min(topk, c + 1)
+ * and min(topk + 2 extra, c + 1) blocks.
+ *
+ * Buffers of the variant are sized by the WIDE shape: `shape` with topk
+ * replaced by W = topk + 2 extra (moba_pooled_wide_shape).  For it
+ * moba_sel_elems, moba_offsets_elems, moba_query_chunk, moba_num_chunks,
+ * moba_gate_workspace_size and moba_attn_workspace_size give the variant's
+ * sizes; moba_rows_elems gives an upper bound of its rows entries (the gate
+ * writes offsets[last] of them). */
+
+/* The wide shape of the variant: *wide = *shape with topk + 2 extra.  Returns
+ * MOBA_ERR_INVALID_ARG for extra < 0 and MOBA_ERR_UNSUPPORTED when
+ * topk + 2 extra > MOBA_MAX_TOPK; host only. */
+MOBA_API moba_status_t moba_pooled_wide_shape(const moba_shape_t* shape, int32_t extra,
+                                              moba_shape_t* wide);
+
+/* Channel-wise max and min of every block's keys.
+ *   k      [batch, seqlen, hkv, head_dim]  dtype     (read)
+ *   maxk   [batch, n, hkv, head_dim]       fp32      (written)
+ *   mink   [batch, n, hkv, head_dim]       fp32      (written)
+ * Exact (no rounding): maxk/mink hold the inputs' own values. */
+MOBA_API moba_status_t moba_block_maxminpool(const moba_shape_t* shape, const void* k, float* maxk,
+                                             float* mink, moba_stream_t stream);
+
+/* The variant's gate.  Scores are fp32 dot products of q with the three pooled
+ * keys.
+ *   q, meank        as for moba_gate_topk                              (read)
+ *   maxk, mink      outputs of moba_block_maxminpool                   (read)
+ *   sel      [batch, seqlen, hq, W] int32 (written): the chosen earlier blocks
+ *            ascending, then the current block, then -1
+ *   offsets, rows   as for moba_gate_topk, for the wide shape          (written)
+ *   ws       >= moba_gate_workspace_size(wide) bytes of device scratch */
+MOBA_API moba_status_t moba_gate_pooled(const moba_shape_t* shape, int32_t extra, const void* q,
+                                        const float* meank, const float* maxk, const float* mink,
+                                        int32_t* sel, int32_t* offsets, int32_t* rows, void* ws,
+                                        size_t ws_bytes, moba_stream_t stream);
+
+/* Attention over the variant's selections: the kernels of moba_attn_fwd for
+ * the wide shape, plus one kernel per pass that marks the partial-result slots
+ * of rows that chose fewer blocks as empty before the merge.
+ *   arguments as for moba_attn_fwd; sel, offsets, rows from moba_gate_pooled
+ *   ws   >= moba_attn_workspace_size(wide) bytes; first int32 = status word */
+MOBA_API moba_status_t moba_attn_fwd_pooled(const moba_shape_t* shape, int32_t extra, const void* q,
+                                            const void* k, const void* v, const int32_t* sel,
+                                            const int32_t* offsets, const int32_t* rows, void* out,
+                                            float* lse, void* ws, size_t ws_bytes,
+                                            moba_stream_t stream);
+
 /* ---- diagnostics ------------------------------------------------------- */
 
 /* Static description of a status code. */

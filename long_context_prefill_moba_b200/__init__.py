@@ -33,6 +33,8 @@ __all__ = [
     "moba_status_string", "moba_last_launch_count", "moba_gate_topk_noalloc", "MobaLayer", "moba_forward",
     "moba_prefill_host_workspace_size", "moba_prefill_host", "MobaHostLayer",
     "moba_attn_bwd_workspace_size", "moba_attn_bwd", "moba_attention",
+    "moba_pooled_wide_shape", "moba_block_maxminpool", "moba_gate_pooled", "moba_attn_fwd_pooled",
+    "MobaPooledLayer", "moba_forward_pooled",
     "MOBA_BF16", "MOBA_F32", "EXPORTED_SYMBOLS",
 ]
 
@@ -49,7 +51,8 @@ EXPORTED_SYMBOLS = [
     "moba_gate_topk", "moba_attn_fwd", "moba_status_string", "moba_last_cuda_error",
     "moba_last_launch_count", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait",
     "moba_prefill_host_workspace_size", "moba_prefill_host", "moba_attn_bwd_workspace_size",
-    "moba_attn_bwd",
+    "moba_attn_bwd", "moba_pooled_wide_shape", "moba_block_maxminpool", "moba_gate_pooled",
+    "moba_attn_fwd_pooled",
 ]
 
 
@@ -115,6 +118,15 @@ def load_library(path: str = LIB_PATH):
     L.moba_prefill_host_workspace_size.restype = sz
     L.moba_prefill_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.moba_prefill_host.restype = st
+    i32 = ctypes.c_int32
+    L.moba_pooled_wide_shape.argtypes = [P, i32, P]
+    L.moba_pooled_wide_shape.restype = st
+    L.moba_block_maxminpool.argtypes = [P, vp, vp, vp, vp]
+    L.moba_block_maxminpool.restype = st
+    L.moba_gate_pooled.argtypes = [P, i32] + [vp] * 8 + [sz, vp]
+    L.moba_gate_pooled.restype = st
+    L.moba_attn_fwd_pooled.argtypes = [P, i32] + [vp] * 9 + [sz, vp]
+    L.moba_attn_fwd_pooled.restype = st
     L.moba_status_string.argtypes = [st]
     L.moba_status_string.restype = ctypes.c_char_p
     L.moba_last_cuda_error.argtypes = []
@@ -235,6 +247,32 @@ def moba_attn_bwd(shape, q, k, v, out, dout, lse, sel, offsets, rows, dq, dk, dv
            "moba_attn_bwd")
 
 
+def moba_pooled_wide_shape(shape, extra) -> MobaShape:
+    """The shape that sizes the pooled-gate variant's buffers: topk + 2 * extra."""
+    wide = MobaShape()
+    _check(lib().moba_pooled_wide_shape(_s(shape), int(extra), _s(wide)), "moba_pooled_wide_shape")
+    return wide
+
+
+def moba_block_maxminpool(shape, k, maxk, mink, stream=None):
+    _check(lib().moba_block_maxminpool(_s(shape), _ptr(k), _ptr(maxk), _ptr(mink), _stream(stream)),
+           "moba_block_maxminpool")
+
+
+def moba_gate_pooled(shape, extra, q, meank, maxk, mink, sel, offsets, rows, ws, stream=None):
+    _check(lib().moba_gate_pooled(_s(shape), int(extra), _ptr(q), _ptr(meank), _ptr(maxk), _ptr(mink),
+                                  _ptr(sel), _ptr(offsets), _ptr(rows), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)),
+           "moba_gate_pooled")
+
+
+def moba_attn_fwd_pooled(shape, extra, q, k, v, sel, offsets, rows, out, lse, ws, stream=None):
+    _check(lib().moba_attn_fwd_pooled(_s(shape), int(extra), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
+                                      _ptr(offsets), _ptr(rows), _ptr(out), _ptr(lse), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)),
+           "moba_attn_fwd_pooled")
+
+
 class MobaHostLayer:
     """One MoBA layer shape served from host buffers (moba_prefill_host): the
     device workspace is allocated once; ``forward`` enqueues the copies and the
@@ -336,6 +374,79 @@ class MobaLayer:
     def meank_view(self):
         s = self.shape
         return self.meank.view(s.batch, moba_num_blocks(s), s.hkv, s.head_dim)
+
+
+class MobaPooledLayer:
+    """Buffers of one layer shape for the gate variant that also routes the top
+    `extra` blocks by max- and by min-pooled keys, and its four steps:
+    mean-pool, max/min-pool, the three-ranking gate and the attention.  Buffers
+    sized by the wide shape (topk + 2 * extra); ``rows`` holds an upper bound
+    of entries, of which the gate fills ``offsets[-1]``."""
+
+    def __init__(self, batch, seqlen, hq, hkv, head_dim, block, topk, extra, dtype="bf16", scale=None,
+                 query_chunk=0, device="cuda"):
+        self.shape = make_shape(batch, seqlen, hq, hkv, head_dim, block, topk, dtype, scale, query_chunk)
+        self.extra = int(extra)
+        self.wide = moba_pooled_wide_shape(self.shape, self.extra)
+        dev = torch.device(device)
+        self.device = dev
+        i32, f32 = torch.int32, torch.float32
+        w = self.wide
+        self.meank = torch.empty(moba_meank_elems(w), dtype=f32, device=dev)
+        self.maxk = torch.empty_like(self.meank)
+        self.mink = torch.empty_like(self.meank)
+        self.sel = torch.empty(moba_sel_elems(w), dtype=i32, device=dev)
+        self.offsets = torch.empty(moba_offsets_elems(w), dtype=i32, device=dev)
+        self.rows = torch.empty(max(1, moba_rows_elems(w)), dtype=i32, device=dev)
+        self.gate_ws = torch.empty(moba_gate_workspace_size(w), dtype=torch.uint8, device=dev)
+        self.attn_ws = torch.empty(moba_attn_workspace_size(w), dtype=torch.uint8, device=dev)
+        self.launches = 0
+
+    @classmethod
+    def from_config(cls, cfg, extra, device="cuda", query_chunk=0):
+        return cls(cfg.batch, cfg.seqlen, cfg.hq, cfg.hkv, cfg.head_dim, cfg.block, cfg.topk, extra,
+                   cfg.dtype, cfg.scale, query_chunk, device)
+
+    def forward(self, q, k, v, out, lse=None, stream=None):
+        s, x = self.shape, self.extra
+        moba_block_meanpool(s, k, self.meank, stream)
+        n = moba_last_launch_count()
+        moba_block_maxminpool(s, k, self.maxk, self.mink, stream)
+        n += moba_last_launch_count()
+        moba_gate_pooled(s, x, q, self.meank, self.maxk, self.mink, self.sel, self.offsets, self.rows,
+                         self.gate_ws, stream)
+        n += moba_last_launch_count()
+        moba_attn_fwd_pooled(s, x, q, k, v, self.sel, self.offsets, self.rows, out, lse, self.attn_ws,
+                             stream)
+        n += moba_last_launch_count()
+        self.launches = n
+        return out
+
+    def device_status(self):
+        torch.cuda.synchronize(self.device)
+        g = self.gate_ws[-256:-252].view(torch.int32).item()
+        a = self.attn_ws[:4].view(torch.int32).item()
+        return g, a
+
+    def sel_view(self):
+        w = self.wide
+        return self.sel.view(w.batch, w.seqlen, w.hq, w.topk)
+
+    def pool_views(self):
+        s = self.shape
+        shp = (s.batch, moba_num_blocks(s), s.hkv, s.head_dim)
+        return self.meank.view(shp), self.maxk.view(shp), self.mink.view(shp)
+
+
+def moba_forward_pooled(q, k, v, block, topk, extra, scale=None, return_lse=False, query_chunk=0):
+    """out (and lse) of one layer with the pooled-gate variant."""
+    b, N, hq, d = q.shape
+    layer = MobaPooledLayer(b, N, hq, k.shape[2], d, block, topk, extra, q.dtype, scale, query_chunk,
+                            q.device)
+    out = torch.empty_like(q)
+    lse = torch.empty(b, hq, N, dtype=torch.float32, device=q.device) if return_lse else None
+    layer.forward(q, k, v, out, lse)
+    return (out, lse) if return_lse else out
 
 
 def moba_forward(q, k, v, block, topk, scale=None, return_lse=False, query_chunk=0):

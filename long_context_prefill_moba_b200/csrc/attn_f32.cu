@@ -60,6 +60,7 @@ __global__ void __launch_bounds__(kWarps * 32) attn_hist_f32_kernel(
   const int ngroups = dm.batch * dm.hkv * dm.n;
   const int32_t* off = offsets + (size_t)ch * ngroups;
   const int p = off[0] + w;
+  if (p >= off[ngroups]) return;   // nrows may be an upper bound (pooled gate)
   int lo = 0, hi = ngroups - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;

@@ -263,6 +263,12 @@ cudaError_t launch_select(const Dims& dm, const void* q, const float* meank, int
 
 }  // namespace
 
+cudaError_t launch_gate_scan(const int32_t* in, int32_t* out, int64_t L, int32_t base,
+                             cudaStream_t stream) {
+  gate_scan_kernel<<<1, kScanThreads, 0, stream>>>(in, out, L, base);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gate(const Dims& dm, int dtype, const void* q, const float* meank, int32_t* sel,
                         int32_t* offsets, int32_t* rows, GateWs ws, cudaStream_t stream,
                         int* launches) {

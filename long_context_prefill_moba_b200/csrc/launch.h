@@ -48,6 +48,19 @@ cudaError_t launch_gate_noalloc(const Dims& dm, int dtype, const void* q, const 
                                 int32_t* sel, int32_t* offsets, int32_t* rows,
                                 cudaStream_t stream, int* launches);
 
+// exclusive prefix sum of in[0..L) plus `base` into out[0..L] (one CTA)
+cudaError_t launch_gate_scan(const int32_t* in, int32_t* out, int64_t L, int32_t base,
+                             cudaStream_t stream);
+
+// gate variant with max- and min-pooled keys (dm.topk = the selection width
+// W = km + 1 + 2 * extra; km = slots of the mean ranking)
+cudaError_t launch_maxminpool(const Dims& dm, int dtype, const void* k, float* maxk, float* mink,
+                              cudaStream_t stream, int* launches);
+cudaError_t launch_gate_pooled(const Dims& dm, int dtype, int km, int extra, const void* q,
+                               const float* meank, const float* maxk, const float* mink, int32_t* sel,
+                               int32_t* offsets, int32_t* rows, GateWs ws, cudaStream_t stream,
+                               int* launches);
+
 struct AttnWs {
   int* status;          // device status word: 0, or MOBA_ERR_TIMEOUT after a bounded wait expired
   float* part_o;        // [b * C * hq * (topk-1), d]  normalised partial outputs
@@ -62,6 +75,13 @@ cudaError_t launch_attn_passes(const Dims& dm, int dtype, const void* q, const v
                                const void* v, const int32_t* sel, const int32_t* offsets,
                                const int32_t* rows, void* out, float* lse, AttnWs ws, int ch_begin,
                                int ch_end, cudaStream_t stream, int* launches);
+
+// the attention step over the pooled gate's selections (rows with fewer
+// chosen blocks than the width allows): launch_attn plus the per-pass fill of
+// the partial slots no historical tile writes
+cudaError_t launch_attn_pooled(const Dims& dm, int dtype, const void* q, const void* k, const void* v,
+                               const int32_t* sel, const int32_t* offsets, const int32_t* rows,
+                               void* out, float* lse, AttnWs ws, cudaStream_t stream, int* launches);
 
 // backward of the attention step: dq, dk, dv (in the input dtype) given dout,
 // the forward's out and lse and the gate's sel/offsets/rows

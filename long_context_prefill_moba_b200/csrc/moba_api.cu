@@ -449,6 +449,88 @@ MOBA_API moba_status_t moba_prefill_host(const moba_shape_t* s, const void* q, c
   return finish(e, launches);
 }
 
+// ---- gate variant with max- and min-pooled keys ------------------------------
+
+MOBA_API moba_status_t moba_pooled_wide_shape(const moba_shape_t* s, int32_t extra, moba_shape_t* wide) {
+  if (wide == nullptr) return MOBA_ERR_INVALID_ARG;
+  moba_status_t st = moba_check_shape(s);
+  if (st != MOBA_OK) return st;
+  if (extra < 0) return MOBA_ERR_INVALID_ARG;
+  if ((int64_t)s->topk + 2 * (int64_t)extra > MOBA_MAX_TOPK) return MOBA_ERR_UNSUPPORTED;
+  moba_shape_t w = *s;
+  w.topk = s->topk + 2 * extra;
+  if ((st = moba_check_shape(&w)) != MOBA_OK) return st;
+  *wide = w;
+  return MOBA_OK;
+}
+
+MOBA_API moba_status_t moba_block_maxminpool(const moba_shape_t* s, const void* k, float* maxk,
+                                             float* mink, moba_stream_t stream) {
+  g_last_launches = 0;
+  moba_status_t st = moba_check_shape(s);
+  if (st != MOBA_OK) return st;
+  if (k == nullptr || maxk == nullptr || mink == nullptr || !aligned16(k) || !aligned16(maxk) ||
+      !aligned16(mink))
+    return MOBA_ERR_INVALID_ARG;
+  int launches = 0;
+  cudaError_t e = moba::launch_maxminpool(make_dims(s), s->dtype, k, maxk, mink, (cudaStream_t)stream,
+                                          &launches);
+  return finish(e, launches);
+}
+
+MOBA_API moba_status_t moba_gate_pooled(const moba_shape_t* s, int32_t extra, const void* q,
+                                        const float* meank, const float* maxk, const float* mink,
+                                        int32_t* sel, int32_t* offsets, int32_t* rows, void* ws,
+                                        size_t ws_bytes, moba_stream_t stream) {
+  g_last_launches = 0;
+  moba_shape_t w;
+  moba_status_t st = moba_pooled_wide_shape(s, extra, &w);
+  if (st != MOBA_OK) return st;
+  if (q == nullptr || meank == nullptr || maxk == nullptr || mink == nullptr || sel == nullptr ||
+      offsets == nullptr || ws == nullptr)
+    return MOBA_ERR_INVALID_ARG;
+  if (rows == nullptr && rows_total(&w) > 0) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(meank) || !aligned16(maxk) || !aligned16(mink) || !aligned4(sel) ||
+      !aligned4(offsets) || (rows != nullptr && !aligned4(rows)) || !aligned16(ws))
+    return MOBA_ERR_INVALID_ARG;
+  if (ws_bytes < moba_gate_workspace_size(&w)) return MOBA_ERR_WORKSPACE;
+  const int64_t L = ngroups_total(&w);
+  moba::GateWs g{static_cast<int32_t*>(ws), static_cast<int32_t*>(ws) + L,
+                 reinterpret_cast<int*>(static_cast<char*>(ws) + align_up(2 * (size_t)L * sizeof(int32_t)))};
+  int launches = 0;
+  cudaError_t e = moba::launch_gate_pooled(make_dims(&w), s->dtype, s->topk - 1, extra, q, meank, maxk,
+                                           mink, sel, offsets, rows, g, (cudaStream_t)stream, &launches);
+  return finish(e, launches);
+}
+
+MOBA_API moba_status_t moba_attn_fwd_pooled(const moba_shape_t* s, int32_t extra, const void* q,
+                                            const void* k, const void* v, const int32_t* sel,
+                                            const int32_t* offsets, const int32_t* rows, void* out,
+                                            float* lse, void* ws, size_t ws_bytes, moba_stream_t stream) {
+  g_last_launches = 0;
+  moba_shape_t w;
+  moba_status_t st = moba_pooled_wide_shape(s, extra, &w);
+  if (st != MOBA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || sel == nullptr || offsets == nullptr ||
+      out == nullptr || ws == nullptr)
+    return MOBA_ERR_INVALID_ARG;
+  if (rows == nullptr && rows_total(&w) > 0) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(sel) ||
+      !aligned4(offsets) || (rows != nullptr && !aligned4(rows)) || !aligned16(ws) ||
+      (lse != nullptr && !aligned4(lse)))
+    return MOBA_ERR_INVALID_ARG;
+  if (ws_bytes < moba_attn_workspace_size(&w)) return MOBA_ERR_WORKSPACE;
+  AttnLayout L = attn_layout(&w);
+  char* base = static_cast<char*>(ws);
+  moba::AttnWs a{reinterpret_cast<int*>(base + L.status), reinterpret_cast<float*>(base + L.part_o),
+                 reinterpret_cast<float*>(base + L.part_lse),
+                 reinterpret_cast<int32_t*>(base + L.tile_start)};
+  int launches = 0;
+  cudaError_t e = moba::launch_attn_pooled(make_dims(&w), s->dtype, q, k, v, sel, offsets, rows, out,
+                                           lse, a, (cudaStream_t)stream, &launches);
+  return finish(e, launches);
+}
+
 MOBA_API const char* moba_status_string(moba_status_t st) {
   switch (st) {
     case MOBA_OK: return "MOBA_OK";

@@ -151,12 +151,49 @@ def test_status_strings(L):
 
 
 def test_library_missing_fails_loudly(tmp_path):
-    import importlib
-    mod = importlib.reload(M)
-    saved = mod._lib
+    saved = M._lib
     try:
-        mod._lib = None
+        M._lib = None
         with pytest.raises(RuntimeError, match="no CPU fallback"):
-            mod.load_library(str(tmp_path / "libmoba.so"))
+            M.load_library(str(tmp_path / "libmoba.so"))
     finally:
-        mod._lib = saved
+        M._lib = saved
+
+
+def test_pooled_gate_wide_shape_sizes_and_validation(L):
+    s = shape(batch=1, seqlen=4096, hq=4, hkv=2, block=256, topk=4)
+    w = M.moba_pooled_wide_shape(s, 2)
+    assert w.topk == 8
+    assert [getattr(w, f) for f, _ in M.MobaShape._fields_ if f != "topk"] == \
+        [getattr(s, f) for f, _ in M.MobaShape._fields_ if f != "topk"]
+    assert M.moba_pooled_wide_shape(s, 0).topk == 4
+    # rows: an upper bound, every row with at most min(W - 1, c) earlier blocks
+    assert M.moba_rows_elems(w) == sum(min(7, t // 256) for t in range(4096)) * 4
+    assert M.moba_sel_elems(w) == 4096 * 4 * 8
+    for extra, status in ((-1, 1), (7, 2)):                  # 4 + 2 * 7 > MOBA_MAX_TOPK
+        with pytest.raises(M.MobaError) as e:
+            M.moba_pooled_wide_shape(s, extra)
+        assert e.value.status == status
+    assert M.moba_pooled_wide_shape(shape(topk=16), 0).topk == 16
+
+    fake = ctypes.c_void_p(1 << 20)          # never dereferenced: validation fails first
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    P = ctypes.byref(s)
+    big = 1 << 40
+    assert L.moba_block_maxminpool(P, fake, None, fake, None) == 1
+    assert L.moba_block_maxminpool(P, fake, fake, odd, None) == 1
+    # moba_gate_pooled(shape, extra, q, meank, maxk, mink, sel, offsets, rows, ws, ws_bytes, stream)
+    assert L.moba_gate_pooled(P, 2, *[fake] * 8, 16, None) == 3
+    assert L.moba_gate_pooled(P, 2, *[fake] * 8, M.moba_gate_workspace_size(w) - 1, None) == 3
+    assert L.moba_gate_pooled(P, -1, *[fake] * 8, big, None) == 1
+    assert L.moba_gate_pooled(P, 7, *[fake] * 8, big, None) == 2
+    assert L.moba_gate_pooled(P, 2, fake, fake, None, fake, fake, fake, fake, fake, big, None) == 1
+    # moba_attn_fwd_pooled(shape, extra, q, k, v, sel, offsets, rows, out, lse, ws, ws_bytes, stream)
+    assert L.moba_attn_fwd_pooled(P, 2, *[fake] * 7, None, fake, 16, None) == 3
+    assert L.moba_attn_fwd_pooled(P, 2, *[fake] * 7, None, fake, M.moba_attn_workspace_size(w) - 1,
+                                  None) == 3
+    assert L.moba_attn_fwd_pooled(P, 2, fake, fake, odd, *[fake] * 4, None, fake, big, None) == 1
+    assert L.moba_attn_fwd_pooled(P, 9, *[fake] * 7, None, fake, big, None) == 2
+    assert L.moba_last_launch_count() == 0
+    # the attention workspace of the variant holds W - 1 partial slots per row
+    assert M.moba_attn_workspace_size(w) > M.moba_attn_workspace_size(s)
