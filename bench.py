@@ -303,6 +303,69 @@ def backward_bench(cfg, steps, warmup):
                       "device_status": status}), flush=True)
 
 
+def pooled_gate_bench(cfg, extra, steps, warmup):
+    """One JSON line: the layer with the gate variant that also routes the top
+    `extra` blocks by max- and min-pooled keys (mean-pool, max/min-pool, the
+    three-ranking gate, attention at width topk + 2 extra) beside the plain
+    layer on the same inputs, inputs resident in HBM, CUDA events on the
+    stream.  Algorithmic FLOPs count the pairs the variant's gate routed:
+    4 d (B x routed (row, earlier block) pairs + the causal current blocks)."""
+    import long_context_prefill_moba_b200 as M
+    M.load_library()
+    dev = torch.device("cuda", 0)
+    q, k, v = S.gen_q(cfg, dev), S.gen_k(cfg, dev), S.gen_v(cfg, dev)
+    out = torch.empty_like(q)
+    pooled = M.MobaPooledLayer.from_config(cfg, extra, dev)
+    plain = M.MobaLayer.from_config(cfg, dev)
+
+    def timed(layer):
+        for _ in range(warmup):
+            layer.forward(q, k, v, out)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            layer.forward(q, k, v, out)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    ms_plain = timed(plain)
+    ms_pooled = timed(pooled)
+    # the variant's stages, once more with events between the calls
+    sh, x = pooled.shape, pooled.extra
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    ev[0].record()
+    M.moba_block_meanpool(sh, k, pooled.meank)
+    ev[1].record()
+    M.moba_block_maxminpool(sh, k, pooled.maxk, pooled.mink)
+    ev[2].record()
+    M.moba_gate_pooled(sh, x, q, pooled.meank, pooled.maxk, pooled.mink, pooled.sel, pooled.offsets,
+                       pooled.rows, pooled.gate_ws)
+    ev[3].record()
+    M.moba_attn_fwd_pooled(sh, x, q, k, v, pooled.sel, pooled.offsets, pooled.rows, out, None,
+                           pooled.attn_ws)
+    ev[4].record()
+    torch.cuda.synchronize()
+    stages = {n: ev[i].elapsed_time(ev[i + 1]) for i, n in enumerate(("meanpool", "maxminpool", "gate",
+                                                                      "attention"))}
+    routed = int(pooled.offsets[-1].item())
+    cur_pairs = 0
+    for c in range(cfg.nblocks):
+        L = min(cfg.seqlen, (c + 1) * cfg.block) - c * cfg.block
+        cur_pairs += L * (L + 1) // 2
+    flops = 4.0 * cfg.head_dim * (routed * cfg.block + cur_pairs * cfg.batch * cfg.hq)
+    peaks, _ = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    print(json.dumps({"mode": "pooled_gate", "workload": cfg.name, "seqlen": cfg.seqlen, "topk": cfg.topk,
+                      "extra": extra, "width": cfg.topk + 2 * extra, "ms_per_layer": ms_pooled,
+                      "ms_per_layer_plain_gate": ms_plain, "stage_ms": stages,
+                      "routed_pairs": routed, "routed_pairs_plain_gate": M.moba_rows_elems(plain.shape),
+                      "tflops": flops / ms_pooled / 1e9, "frac_of_sustained_peak": flops / ms_pooled / 1e9 / peak,
+                      "steps": steps, "warmup": warmup, "gpu_launches_per_step": pooled.launches,
+                      "device_status": list(pooled.device_status())}), flush=True)
+
+
 def speedup_curve(seqlens, reps=2):
     """One JSON line per sequence length: the MoBA layer (mean-pool + gate +
     attention through the C ABI) against dense causal attention on the same
@@ -378,6 +441,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--backward", action="store_true",
                     help="time the attention backward (moba_attn_bwd) instead; prints its own JSON line")
+    ap.add_argument("--pooled-gate", type=int, default=None, metavar="EXTRA",
+                    help="time the gate variant that adds the top EXTRA blocks by max- and "
+                         "min-pooled keys, beside the plain layer")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
@@ -388,6 +454,9 @@ def main():
     args = ap.parse_args()
     if args.speedup_curve:
         speedup_curve([int(x) for x in args.curve_seqlens.split(",")])
+        return
+    if args.pooled_gate is not None:
+        pooled_gate_bench(S.get_config(args.config), args.pooled_gate, args.steps, args.warmup)
         return
     if args.backward:
         backward_bench(S.get_config(args.config), args.steps, args.warmup)

@@ -14,7 +14,11 @@ Functions with the names of the C entry points:
     moba_attn_fwd(shape, q, k, v, sel, offsets, rows, out, lse, ws)
 
 plus ``MobaLayer`` (owns the intermediate buffers of one shape and runs the
-three steps) and ``moba_forward`` (allocating convenience call).
+three steps) and ``moba_forward`` (allocating convenience call), the backward
+(``moba_attn_bwd``, ``moba_attention``), the host-buffer layer
+(``moba_prefill_host``, ``MobaHostLayer``) and the gate variant with max- and
+min-pooled keys (``moba_block_maxminpool``, ``moba_gate_pooled``,
+``moba_attn_fwd_pooled``, ``MobaPooledLayer``, ``moba_forward_pooled``).
 """
 from __future__ import annotations
 
