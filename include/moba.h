@@ -303,7 +303,10 @@ MOBA_API moba_status_t moba_gate_pooled(const moba_shape_t* shape, int32_t extra
  * the wide shape, plus one kernel per pass that marks the partial-result slots
  * of rows that chose fewer blocks as empty before the merge.
  *   arguments as for moba_attn_fwd; sel, offsets, rows from moba_gate_pooled
- *   ws   >= moba_attn_workspace_size(wide) bytes; first int32 = status word */
+ *   ws   >= moba_attn_workspace_size(wide) bytes; first int32 = status word
+ * The variant's backward is moba_attn_bwd called with the wide shape and this
+ * gate's sel, offsets and rows: its kernels read variable-length selections
+ * through them (rows entries up to offsets[last]). */
 MOBA_API moba_status_t moba_attn_fwd_pooled(const moba_shape_t* shape, int32_t extra, const void* q,
                                             const void* k, const void* v, const int32_t* sel,
                                             const int32_t* offsets, const int32_t* rows, void* out,

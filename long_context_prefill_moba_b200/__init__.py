@@ -426,6 +426,18 @@ class MobaPooledLayer:
         self.launches = n
         return out
 
+    def backward(self, q, k, v, out, lse, dout, dq, dk, dv, stream=None):
+        """dq, dk, dv of the last forward's attention given dout, its selection
+        held fixed: moba_attn_bwd at the wide shape (its kernels read the
+        variable-length selections through sel, offsets and rows)."""
+        if getattr(self, "bwd_ws", None) is None:
+            self.bwd_ws = torch.empty(moba_attn_bwd_workspace_size(self.wide), dtype=torch.uint8,
+                                      device=self.device)
+        moba_attn_bwd(self.wide, q, k, v, out, dout, lse, self.sel, self.offsets, self.rows, dq, dk, dv,
+                      self.bwd_ws, stream)
+        self.launches = moba_last_launch_count()
+        return dq, dk, dv
+
     def device_status(self):
         torch.cuda.synchronize(self.device)
         g = self.gate_ws[-256:-252].view(torch.int32).item()

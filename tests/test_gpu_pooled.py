@@ -147,3 +147,26 @@ def test_pooled_extra_zero_selects_like_the_plain_gate(cuda_device):
     assert rows_same.mean() > 0.98
     d = (out.float() - out_p.float()).abs().cpu().numpy()[rows_same].max()
     assert d <= out_tol(cfg)
+
+
+@pytest.mark.parametrize("name", ["bf16_d128_multipass", "bf16_d64_mqa", "f32_wide"])
+def test_pooled_backward_with_the_selection_fixed(cuda_device, name):
+    # the variant's backward is moba_attn_bwd at the wide shape; reference: the
+    # backward oracle with the GPU gate's (variable-length) selection
+    from oracle import moba_backward as OB
+    cfg, extra, chunk = CASES[name]
+    layer, out, lse = run_pooled(cfg, extra, chunk)
+    dev = torch.device("cuda:0")
+    q, k, v, dout = S.gen_q(cfg, dev), S.gen_k(cfg, dev), S.gen_v(cfg, dev), S.gen_dout(cfg, dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    layer.backward(q, k, v, out, lse, dout, dq, dk, dv)
+    torch.cuda.synchronize()
+    assert layer.bwd_ws[:4].view(torch.int32).item() == 0 and layer.launches > 0
+    sel = layer.sel_view().cpu().numpy()
+    rq, rk, rv, _ = OB.moba_backward(S.gen_q(cfg), S.gen_k(cfg), S.gen_v(cfg), S.gen_dout(cfg), cfg.block,
+                                     cfg.topk + 2 * extra, cfg.softmax_scale, sel=sel)
+    for name_, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        err = float(np.abs(cpu(got).numpy() - ref).max())
+        bound = (3e-2 if cfg.dtype == "bf16" else 2e-4) * max(1.0, float(np.abs(ref).max()))
+        print(name, name_, "max abs err", err, "max |ref|", float(np.abs(ref).max()))
+        assert err <= bound, (name, name_, err)
