@@ -96,3 +96,33 @@ def test_every_earlier_block_selected_is_dense_causal():
     tq, tk, tv = (torch.tensor(x).transpose(1, 2) for x in (q, k.repeat(2, 2), v.repeat(2, 2)))
     ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=0.4)
     assert np.abs(out - ref.transpose(1, 2).numpy()).max() <= 1e-12
+
+
+@pytest.mark.parametrize("seed,N,B,Hq,Hkv,topk,extra", [
+    (0, 37, 5, 4, 2, 3, 1), (1, 50, 7, 2, 1, 2, 2), (2, 64, 8, 3, 3, 1, 3), (3, 41, 6, 4, 1, 4, 1),
+])
+def test_layer_is_masked_attention_over_its_selections(seed, N, B, Hq, Hkv, topk, extra):
+    # an independent formulation for rows with any number of selected blocks: fp64
+    # SDPA (a library routine) with the boolean mask "key u is in a selected block
+    # and u <= t" built from the layer's own selections
+    rng = np.random.default_rng(seed)
+    d = 6
+    q = rng.standard_normal((1, N, Hq, d))
+    k = rng.standard_normal((1, N, Hkv, d)) + rng.standard_normal((1, (N + B - 1) // B, Hkv, d)).repeat(B, 1)[:, :N]
+    v = rng.standard_normal((1, N, Hkv, d))
+    out, lse, sels = P.moba_pooled_layer(q, k, v, B, topk, extra, 0.35)
+    G = Hq // Hkv
+    mask = torch.zeros(1, Hq, N, N, dtype=torch.bool)
+    for (_, t, h), sel in sels.items():
+        for j in sel:
+            mask[0, h, t, j * B: min(N, (j + 1) * B)] = True
+    mask &= torch.ones(N, N, dtype=torch.bool).tril()
+    tq = torch.tensor(q).transpose(1, 2)
+    tk, tv = (torch.tensor(x).repeat_interleave(G, 2).transpose(1, 2) for x in (k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=0.35)
+    assert np.abs(out - ref.transpose(1, 2).numpy()).max() <= 1e-12
+    z = 0.35 * torch.einsum("bhtd,bhud->bhtu", tq, tk).masked_fill(~mask, float("-inf"))
+    assert np.abs(lse - torch.logsumexp(z, -1).numpy()).max() <= 1e-12
+    # some rows attend fewer blocks than the width allows (the rankings overlap)
+    widths = [len(s) for (_, t, _), s in sels.items() if t // B + 1 > topk + 2 * extra]
+    assert widths and min(widths) >= topk and max(widths) <= topk + 2 * extra
