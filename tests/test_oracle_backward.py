@@ -109,3 +109,29 @@ def test_zero_upstream_gradient_gives_zero(topk):
     q, k, v, do = rand_inputs(1, 30, 2, 1, 4, 7)
     dq, dk, dv, _ = OB.moba_backward(q, k, v, np.zeros_like(do), 6, topk, 0.5)
     assert not dq.any() and not dk.any() and not dv.any()
+
+
+def test_variable_length_selections_of_the_pooled_gate():
+    # the gate variant with max/min-pooled keys gives rows different numbers of
+    # blocks; the backward oracle with such a frozen selection equals fp64
+    # autograd of attention under the per-head mask built from it, and its
+    # dense-mask formulation
+    from oracle import moba_pooled_gate as P
+    b, N, hq, hkv, d, B, topk, extra, scale = 1, 48, 4, 2, 8, 6, 2, 2, 0.45
+    q, k, v, do = rand_inputs(b, N, hq, hkv, d, 3)
+    _, _, sels = P.moba_pooled_layer(q, k, v, B, topk, extra, scale)
+    W = topk + 2 * extra
+    sel = np.full((b, N, hq, W), -1, dtype=np.int64)
+    mask = np.zeros((hq, N, N), dtype=bool)
+    for (_, t, h), js in sels.items():
+        sel[0, t, h, :len(js)] = js
+        for j in js:
+            mask[h, t, j * B:min(N, (j + 1) * B)] = True
+    mask &= np.tril(np.ones((N, N), dtype=bool))
+    assert len({len(js) for js in sels.values()}) > 2              # the row widths do vary
+    dq, dk, dv, _ = OB.moba_backward(q, k, v, do, B, W, scale, sel=sel)
+    rq, rk, rv = torch_attention_grads(q, k, v, do, mask, scale)
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        assert np.abs(got - ref).max() <= 1e-12
+    for got, ref in zip((dq, dk, dv), OB.moba_backward_dense(q, k, v, do, sel, B, scale)):
+        assert np.abs(got - ref).max() <= 1e-12
