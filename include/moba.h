@@ -126,6 +126,19 @@ MOBA_API int64_t moba_rows_elems(const moba_shape_t* shape);
 MOBA_API size_t moba_gate_workspace_size(const moba_shape_t* shape);
 MOBA_API size_t moba_attn_workspace_size(const moba_shape_t* shape);
 
+/* The scratch of one layer's gate and attention as one allocation:
+ * moba_gate_workspace_size + moba_attn_workspace_size (both multiples of 256).
+ * Pass ws to moba_gate_topk and ws + moba_gate_workspace_size(shape) to
+ * moba_attn_fwd.  0 for an invalid shape. */
+MOBA_API size_t moba_workspace_size(const moba_shape_t* shape);
+
+/* Capacity the rows array needs: an upper bound of the entries any gate
+ * writes for this shape, batch * hq * sum_t min(topk-1, t / block).  For the
+ * plain gate it is the exact count (moba_rows_elems); for the pooled variant's
+ * wide shape the gate fills offsets[last] <= capacity entries.  -1 for an
+ * invalid shape. */
+MOBA_API int64_t moba_rows_capacity(const moba_shape_t* shape);
+
 /* ---- the three steps --------------------------------------------------- */
 
 /* Block mean-pool ([summary] §3 "Affinity Scoring": the block representation

@@ -38,7 +38,7 @@ __all__ = [
     "moba_prefill_host_workspace_size", "moba_prefill_host", "MobaHostLayer",
     "moba_attn_bwd_workspace_size", "moba_attn_bwd", "moba_attention",
     "moba_pooled_wide_shape", "moba_block_maxminpool", "moba_gate_pooled", "moba_attn_fwd_pooled",
-    "MobaPooledLayer", "moba_forward_pooled",
+    "MobaPooledLayer", "moba_forward_pooled", "moba_workspace_size", "moba_rows_capacity",
     "MOBA_BF16", "MOBA_F32", "EXPORTED_SYMBOLS",
 ]
 
@@ -56,7 +56,7 @@ EXPORTED_SYMBOLS = [
     "moba_last_launch_count", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait",
     "moba_prefill_host_workspace_size", "moba_prefill_host", "moba_attn_bwd_workspace_size",
     "moba_attn_bwd", "moba_pooled_wide_shape", "moba_block_maxminpool", "moba_gate_pooled",
-    "moba_attn_fwd_pooled",
+    "moba_attn_fwd_pooled", "moba_workspace_size", "moba_rows_capacity",
 ]
 
 
@@ -96,10 +96,10 @@ def load_library(path: str = LIB_PATH):
     P = ctypes.POINTER(MobaShape)
     vp, i64, sz, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
     for name in ("moba_num_blocks", "moba_query_chunk", "moba_num_chunks", "moba_meank_elems",
-                 "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems"):
+                 "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems", "moba_rows_capacity"):
         getattr(L, name).argtypes = [P]
         getattr(L, name).restype = i64
-    for name in ("moba_gate_workspace_size", "moba_attn_workspace_size"):
+    for name in ("moba_gate_workspace_size", "moba_attn_workspace_size", "moba_workspace_size"):
         getattr(L, name).argtypes = [P]
         getattr(L, name).restype = sz
     L.moba_check_shape.argtypes = [P]
@@ -166,6 +166,8 @@ def moba_offsets_elems(shape) -> int: return lib().moba_offsets_elems(_s(shape))
 def moba_rows_elems(shape) -> int: return lib().moba_rows_elems(_s(shape))
 def moba_gate_workspace_size(shape) -> int: return lib().moba_gate_workspace_size(_s(shape))
 def moba_attn_workspace_size(shape) -> int: return lib().moba_attn_workspace_size(_s(shape))
+def moba_workspace_size(shape) -> int: return lib().moba_workspace_size(_s(shape))
+def moba_rows_capacity(shape) -> int: return lib().moba_rows_capacity(_s(shape))
 def moba_status_string(status: int) -> str: return lib().moba_status_string(status).decode()
 def moba_last_launch_count() -> int: return lib().moba_last_launch_count()
 

@@ -171,6 +171,13 @@ MOBA_API size_t moba_attn_workspace_size(const moba_shape_t* s) {
   if (moba_check_shape(s) != MOBA_OK) return 0;
   return attn_layout(s).total;
 }
+MOBA_API size_t moba_workspace_size(const moba_shape_t* s) {
+  if (moba_check_shape(s) != MOBA_OK) return 0;
+  return moba_gate_workspace_size(s) + moba_attn_workspace_size(s);
+}
+MOBA_API int64_t moba_rows_capacity(const moba_shape_t* s) {
+  return moba_check_shape(s) == MOBA_OK ? rows_total(s) : -1;
+}
 
 MOBA_API moba_status_t moba_block_meanpool(const moba_shape_t* s, const void* k, float* meank,
                                            moba_stream_t stream) {

@@ -197,3 +197,15 @@ def test_pooled_gate_wide_shape_sizes_and_validation(L):
     assert L.moba_last_launch_count() == 0
     # the attention workspace of the variant holds W - 1 partial slots per row
     assert M.moba_attn_workspace_size(w) > M.moba_attn_workspace_size(s)
+
+
+def test_one_allocation_workspace_and_rows_capacity(L):
+    for s in (shape(), shape(dtype="f32", head_dim=64, seqlen=4096, block=256),
+              shape(batch=2, seqlen=1000, hq=4, hkv=2, block=96, topk=3)):
+        g, a = M.moba_gate_workspace_size(s), M.moba_attn_workspace_size(s)
+        assert M.moba_workspace_size(s) == g + a and g % 256 == 0 and a % 256 == 0
+        assert M.moba_rows_capacity(s) == M.moba_rows_elems(s)
+    w = M.moba_pooled_wide_shape(shape(seqlen=4096, block=256, topk=4), 3)
+    assert M.moba_rows_capacity(w) == sum(min(9, t // 256) for t in range(4096)) * 32
+    bad = shape(hq=5, hkv=2)
+    assert M.moba_workspace_size(bad) == 0 and M.moba_rows_capacity(bad) == -1
