@@ -326,6 +326,32 @@ MOBA_API moba_status_t moba_attn_fwd_pooled(const moba_shape_t* shape, int32_t e
                                             float* lse, void* ws, size_t ws_bytes,
                                             moba_stream_t stream);
 
+/* ---- index validation ---------------------------------------------------- */
+
+/* Checks the query-per-block index on the device before an attention or
+ * backward call uses it (an index from another gate, or a changed gate; the
+ * paper has no counterpart).  The attention kernels index K, V, partials and
+ * outputs with these values unchecked.
+ *   shape    as for the gate that wrote the index (the wide shape for the
+ *            pooled variant)
+ *   exact    nonzero: every sel row holds exactly min(topk, c + 1) blocks (the
+ *            plain gate); 0: between 1 and min(topk, c + 1) (the pooled variant)
+ *   sel, offsets   (read; rewritten only if a check fails)
+ *   rows     moba_rows_capacity(shape) entries                   (read)
+ *   status   device int32                                        (written)
+ * Checks: each sel row strictly ascending in [0, c] with c (the query's block)
+ * last, then -1; offsets[0] = 0, non-decreasing, offsets[last] <= the rows
+ * capacity; every rows entry a row id of the shape whose batch entry, kv head
+ * and pass are those of its group (pass, b, g, j), with j < its block and j in
+ * its sel row.  Duplicate rows entries are not detected.  After the stream
+ * completes, *status is 0, or MOBA_ERR_INTERNAL if a check failed; then the
+ * index has been made inert (offsets all 0, every sel row {c, -1, ...}), so
+ * a later moba_attn_fwd / moba_attn_bwd reads no invalid index (its outputs
+ * are then not meaningful).  Nothing faults or traps. */
+MOBA_API moba_status_t moba_check_index(const moba_shape_t* shape, int32_t exact, int32_t* sel,
+                                        int32_t* offsets, const int32_t* rows, int* status,
+                                        moba_stream_t stream);
+
 /* ---- diagnostics ------------------------------------------------------- */
 
 /* Static description of a status code. */

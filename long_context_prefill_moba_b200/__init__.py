@@ -39,7 +39,7 @@ __all__ = [
     "moba_attn_bwd_workspace_size", "moba_attn_bwd", "moba_attention",
     "moba_pooled_wide_shape", "moba_block_maxminpool", "moba_gate_pooled", "moba_attn_fwd_pooled",
     "MobaPooledLayer", "moba_forward_pooled", "moba_workspace_size", "moba_rows_capacity",
-    "MOBA_BF16", "MOBA_F32", "EXPORTED_SYMBOLS",
+    "moba_check_index", "MOBA_BF16", "MOBA_F32", "EXPORTED_SYMBOLS",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -56,7 +56,7 @@ EXPORTED_SYMBOLS = [
     "moba_last_launch_count", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait",
     "moba_prefill_host_workspace_size", "moba_prefill_host", "moba_attn_bwd_workspace_size",
     "moba_attn_bwd", "moba_pooled_wide_shape", "moba_block_maxminpool", "moba_gate_pooled",
-    "moba_attn_fwd_pooled", "moba_workspace_size", "moba_rows_capacity",
+    "moba_attn_fwd_pooled", "moba_workspace_size", "moba_rows_capacity", "moba_check_index",
 ]
 
 
@@ -131,6 +131,8 @@ def load_library(path: str = LIB_PATH):
     L.moba_gate_pooled.restype = st
     L.moba_attn_fwd_pooled.argtypes = [P, i32] + [vp] * 9 + [sz, vp]
     L.moba_attn_fwd_pooled.restype = st
+    L.moba_check_index.argtypes = [P, i32, vp, vp, vp, vp, vp]
+    L.moba_check_index.restype = st
     L.moba_status_string.argtypes = [st]
     L.moba_status_string.restype = ctypes.c_char_p
     L.moba_last_cuda_error.argtypes = []
@@ -277,6 +279,14 @@ def moba_attn_fwd_pooled(shape, extra, q, k, v, sel, offsets, rows, out, lse, ws
                                       _ptr(offsets), _ptr(rows), _ptr(out), _ptr(lse), _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)),
            "moba_attn_fwd_pooled")
+
+
+def moba_check_index(shape, exact, sel, offsets, rows, status, stream=None):
+    """Validate sel/offsets/rows on the device; `status` a 1-element int32 CUDA
+    tensor that becomes 0, or MOBA_ERR_INTERNAL (5) with the index made inert."""
+    _check(lib().moba_check_index(_s(shape), 1 if exact else 0, _ptr(sel), _ptr(offsets), _ptr(rows),
+                                  _ptr(status), _stream(stream)),
+           "moba_check_index")
 
 
 class MobaHostLayer:

@@ -97,6 +97,12 @@ cudaError_t launch_attn_bwd(const Dims& dm, int dtype, const void* q, const void
                             const int32_t* offsets, const int32_t* rows, void* dq, void* dk, void* dv,
                             BwdWs ws, cudaStream_t stream, int* launches);
 
+// checks of sel / offsets / rows (moba_check_index): the status word becomes
+// MOBA_ERR_INTERNAL on a violation, and the index is then made inert
+cudaError_t launch_index_check(const Dims& dm, int exact, int32_t* sel, int32_t* offsets,
+                               const int32_t* rows, int64_t capacity, int* status, cudaStream_t stream,
+                               int* launches);
+
 // a kernel whose only wait can never complete: it must time out (status word)
 cudaError_t launch_bounded_wait_selftest(int* status, cudaStream_t stream);
 

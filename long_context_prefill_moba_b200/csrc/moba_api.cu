@@ -538,6 +538,22 @@ MOBA_API moba_status_t moba_attn_fwd_pooled(const moba_shape_t* s, int32_t extra
   return finish(e, launches);
 }
 
+MOBA_API moba_status_t moba_check_index(const moba_shape_t* s, int32_t exact, int32_t* sel,
+                                        int32_t* offsets, const int32_t* rows, int* status,
+                                        moba_stream_t stream) {
+  g_last_launches = 0;
+  moba_status_t st = moba_check_shape(s);
+  if (st != MOBA_OK) return st;
+  if (sel == nullptr || offsets == nullptr || status == nullptr) return MOBA_ERR_INVALID_ARG;
+  if (rows == nullptr && rows_total(s) > 0) return MOBA_ERR_INVALID_ARG;
+  if (!aligned4(sel) || !aligned4(offsets) || (rows != nullptr && !aligned4(rows)) || !aligned4(status))
+    return MOBA_ERR_INVALID_ARG;
+  int launches = 0;
+  cudaError_t e = moba::launch_index_check(make_dims(s), exact != 0, sel, offsets, rows, rows_total(s),
+                                           status, (cudaStream_t)stream, &launches);
+  return finish(e, launches);
+}
+
 MOBA_API const char* moba_status_string(moba_status_t st) {
   switch (st) {
     case MOBA_OK: return "MOBA_OK";

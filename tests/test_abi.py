@@ -209,3 +209,17 @@ def test_one_allocation_workspace_and_rows_capacity(L):
     assert M.moba_rows_capacity(w) == sum(min(9, t // 256) for t in range(4096)) * 32
     bad = shape(hq=5, hkv=2)
     assert M.moba_workspace_size(bad) == 0 and M.moba_rows_capacity(bad) == -1
+
+
+def test_check_index_validates_before_launching(L):
+    s = shape(seqlen=4096, block=256)
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    P = ctypes.byref(s)
+    # moba_check_index(shape, exact, sel, offsets, rows, status, stream)
+    assert L.moba_check_index(P, 1, None, fake, fake, fake, None) == 1
+    assert L.moba_check_index(P, 1, fake, fake, fake, None, None) == 1
+    assert L.moba_check_index(P, 1, fake, fake, None, fake, None) == 1     # rows needed: 4096 tokens
+    assert L.moba_check_index(P, 1, fake, odd, fake, fake, None) == 1
+    assert L.moba_check_index(ctypes.byref(shape(hq=5, hkv=2)), 1, fake, fake, fake, fake, None) == 1
+    assert L.moba_last_launch_count() == 0
