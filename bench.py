@@ -48,6 +48,17 @@ def attn_flops(cfg) -> float:
     return 4.0 * cfg.head_dim * algorithmic_pairs(cfg)
 
 
+def routed_flops(cfg, routed_pairs: int) -> float:
+    """Algorithmic FLOPs of a layer whose gate routed `routed_pairs` (row,
+    earlier block) pairs (offsets[last]): B keys per pair plus the causal part
+    of every row's own block.  Earlier blocks are always full ones."""
+    cur = 0
+    for c in range(cfg.nblocks):
+        L = min(cfg.seqlen, (c + 1) * cfg.block) - c * cfg.block
+        cur += L * (L + 1) // 2
+    return 4.0 * cfg.head_dim * (routed_pairs * cfg.block + cur * cfg.batch * cfg.hq)
+
+
 def recorded_traffic(rows_per_layer: int):
     """DRAM bytes of one attention step (moba_attn_fwd) from the committed ncu
     capture (profiles/attn_traffic.json), scaled by the rows the gate routes
@@ -350,11 +361,7 @@ def pooled_gate_bench(cfg, extra, steps, warmup):
     stages = {n: ev[i].elapsed_time(ev[i + 1]) for i, n in enumerate(("meanpool", "maxminpool", "gate",
                                                                       "attention"))}
     routed = int(pooled.offsets[-1].item())
-    cur_pairs = 0
-    for c in range(cfg.nblocks):
-        L = min(cfg.seqlen, (c + 1) * cfg.block) - c * cfg.block
-        cur_pairs += L * (L + 1) // 2
-    flops = 4.0 * cfg.head_dim * (routed * cfg.block + cur_pairs * cfg.batch * cfg.hq)
+    flops = routed_flops(cfg, routed)
     peaks, _ = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     print(json.dumps({"mode": "pooled_gate", "workload": cfg.name, "seqlen": cfg.seqlen, "topk": cfg.topk,
