@@ -52,3 +52,42 @@ def test_backward_formulations_agree(shape):
     rq, rk, rv = OB.moba_backward_dense(q, k, v, do, sel, B, 0.5)
     for a, r in ((dq, rq), (dk, rk), (dv, rv)):
         assert np.abs(a - r).max() <= 1e-9
+
+
+pooled_shapes = st.tuples(
+    st.integers(1, 2),            # batch
+    st.integers(1, 36),           # seqlen
+    st.sampled_from([(1, 1), (2, 1), (4, 2)]),   # (hq, hkv)
+    st.integers(1, 7),            # block
+    st.integers(1, 4),            # topk
+    st.integers(0, 3),            # extra
+    st.integers(0, 2 ** 31 - 1),  # seed
+)
+
+
+@settings(max_examples=40, deadline=None, derandomize=True)
+@given(pooled_shapes)
+def test_pooled_gate_layer_invariants_and_masked_attention(shape):
+    # the gate variant with max/min-pooled keys: every row attends its current
+    # block, a superset of the plain gate's blocks, at most topk + 2 extra blocks,
+    # and its output is softmax attention under the mask of its own selection
+    import torch
+    from oracle import moba_pooled_gate as P
+    b, N, (hq, hkv), B, topk, extra, seed = shape
+    q, k, v, _ = inputs(b, N, hq, hkv, seed)
+    out, lse, sels = P.moba_pooled_layer(q, k, v, B, topk, extra, 0.5)
+    _, _, plain, _ = O.moba_dense(q, k, v, B, topk, 0.5)
+    G = hq // hkv
+    mask = np.zeros((b, hq, N, N), dtype=bool)
+    for (bb, t, h), sel in sels.items():
+        c = t // B
+        assert sel == sorted(set(sel)) and sel[-1] == c
+        assert set(int(x) for x in plain[bb, t, h] if x >= 0) <= set(sel)
+        assert min(topk, c + 1) <= len(sel) <= min(topk + 2 * extra, c + 1)
+        for j in sel:
+            mask[bb, h, t, j * B:min(N, (j + 1) * B)] = True
+    mask &= np.tril(np.ones((N, N), dtype=bool))
+    tq = torch.tensor(q).transpose(1, 2)
+    tk, tv = (torch.tensor(x).repeat_interleave(G, 2).transpose(1, 2) for x in (k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.tensor(mask), scale=0.5)
+    assert np.abs(out - ref.transpose(1, 2).numpy()).max() <= 1e-12
