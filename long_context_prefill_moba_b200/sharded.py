@@ -20,7 +20,10 @@ Partition (``head_shard``), P ranks, G = hq / hkv query heads per kv head:
 Any other (hq, hkv, P) is rejected.
 
 K and V arrive by one broadcast each from the source rank, for the whole
-[b, N, hkv, d] tensors; each rank then copies out its own kv heads.  The
+[b, N, hkv, d] tensors; each rank then copies out its own kv heads.  In the
+backward, each rank computes its query heads' gradients locally and the
+adjoint of the broadcast, a sum-reduce onto the source rank, assembles dK and
+dV (ranks that share a kv head add their contributions).  The
 compute runs in the library's kernels (``MobaLayer``); ``layer_factory``
 exists so the host logic can be exercised on ranks without a GPU.
 """
@@ -88,4 +91,26 @@ class ShardedMobaLayer:
 
     def forward(self, q_local, k, v, out_local, lse_local=None, stream=None):
         k_loc, v_loc = self.broadcast_kv(k, v)
+        self._kv = (k_loc, v_loc)
         return self.layer.forward(q_local, k_loc, v_loc, out_local, lse_local, stream)
+
+    def backward(self, q_local, out_local, lse_local, dout_local, dq_local, dk, dv, stream=None):
+        """Gradients of the last forward, its selection held fixed.  dq_local
+        [b, N, h1-h0, d] receives this rank's query heads' dq.  dk, dv
+        [b, N, hkv, d] receive, on the source rank, the gradients of the
+        broadcast K and V: the adjoint of the broadcast sums every rank's
+        contribution (its kv heads' gradients from its query heads) there,
+        summed in at least fp32; elsewhere they are left as they were."""
+        k_loc, v_loc = self._kv
+        dk_loc, dv_loc = torch.empty_like(k_loc), torch.empty_like(v_loc)
+        self.layer.backward(q_local, k_loc, v_loc, out_local, lse_local, dout_local, dq_local, dk_loc, dv_loc,
+                            stream)
+        # the sum runs in at least fp32 (bf16 partials would round at every add)
+        acc_dtype = torch.promote_types(dk_loc.dtype, torch.float32)
+        for full, part in ((dk, dk_loc), (dv, dv_loc)):
+            acc = torch.zeros(full.shape, dtype=acc_dtype, device=full.device)
+            acc[:, :, self.g0:self.g1] = part
+            dist.reduce(acc, self.src, op=dist.ReduceOp.SUM, group=self.group)
+            if self.rank == self.src:
+                full.copy_(acc)
+        return dq_local, dk, dv

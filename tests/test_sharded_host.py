@@ -3,7 +3,9 @@ partition, and the whole sharded layer on 2 and 4 gloo ranks on the CPU with
 the fp64 oracle standing in for the per-rank GPU layer (a test double passed
 as layer_factory).  K and V exist only on the source rank before the
 broadcast; the ranks' head-sharded outputs, gathered in rank order, must
-equal the unsharded oracle layer exactly."""
+equal the unsharded oracle layer exactly, and so must dq; dK and dV, summed
+onto the source rank by the backward's reduce, must equal the unsharded
+gradients up to the order of the sum."""
 import os
 import socket
 
@@ -53,6 +55,13 @@ class _OracleLayer:
             lse.copy_(torch.from_numpy(l))
         return out
 
+    def backward(self, q, k, v, out, lse, dout, dq, dk, dv, stream=None):
+        from oracle import moba_backward as OB
+        gq, gk, gv, _ = OB.moba_backward(q.numpy(), k.numpy(), v.numpy(), dout.numpy(), self.block, self.topk,
+                                         self.scale)
+        for dst, src in ((dq, gq), (dk, gk), (dv, gv)):
+            dst.copy_(torch.from_numpy(src))
+
 
 def _inputs(b, N, hq, hkv, d):
     g = torch.Generator().manual_seed(5)
@@ -82,8 +91,17 @@ def _worker(rank, world, port, shape, path):
         lses = [torch.empty_like(lse_loc) for _ in range(world)]
         dist.all_gather(outs, out_loc)
         dist.all_gather(lses, lse_loc)
+        # backward: local dq of this rank's heads; dK, dV summed onto the source rank
+        g = torch.Generator().manual_seed(9)
+        dout = torch.randn(b, N, hq, d, generator=g, dtype=torch.float64)
+        dq_loc = torch.empty_like(q_loc)
+        dk, dv = torch.empty(b, N, hkv, d, dtype=torch.float64), torch.empty(b, N, hkv, d, dtype=torch.float64)
+        layer.backward(q_loc, out_loc, lse_loc, dout[:, :, layer.h0:layer.h1].contiguous(), dq_loc, dk, dv)
+        dqs = [torch.empty_like(dq_loc) for _ in range(world)]
+        dist.all_gather(dqs, dq_loc)
         if rank == 0:
-            torch.save({"out": torch.cat(outs, 2), "lse": torch.cat(lses, 1)}, path)
+            torch.save({"out": torch.cat(outs, 2), "lse": torch.cat(lses, 1), "dq": torch.cat(dqs, 2),
+                        "dk": dk, "dv": dv, "dout": dout}, path)
     finally:
         dist.destroy_process_group()
 
@@ -112,3 +130,9 @@ def test_sharded_layer_equals_the_unsharded_layer(tmp_path, shape, world):
     out, lse, _, _ = O.moba_dense(q.numpy(), k.numpy(), v.numpy(), B, topk, 0.3)
     assert np.array_equal(got["out"].numpy(), out)
     assert np.array_equal(got["lse"].numpy(), lse)
+    from oracle import moba_backward as OB
+    dq, dk, dv, _ = OB.moba_backward(q.numpy(), k.numpy(), v.numpy(), got["dout"].numpy(), B, topk, 0.3)
+    assert np.array_equal(got["dq"].numpy(), dq)
+    # dK, dV: sums over ranks in another order than the unsharded loop
+    assert np.abs(got["dk"].numpy() - dk).max() <= 1e-12
+    assert np.abs(got["dv"].numpy() - dv).max() <= 1e-12
