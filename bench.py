@@ -210,6 +210,36 @@ class OracleSample:
         return time.perf_counter() - t0, pairs
 
 
+def cpu_baseline_pooled(cfg, extra, budget_s=15.0):
+    """The pooled-gate variant's oracle (oracle/moba_pooled_gate.py) on sampled
+    rows of one kv head: seconds per row, the pools' time, attended pairs."""
+    from oracle import moba_pooled_gate as P
+    smp = OracleSample(cfg)
+    O, np = smp.O, smp.np
+    t0 = time.perf_counter()
+    kmax, kmin = P.max_pool(smp.K, cfg.block), P.min_pool(smp.K, cfg.block)
+    t_pools = smp.t_pool + time.perf_counter() - t0
+    secs, pairs, nrows = 0.0, 0, 0
+    while secs < budget_s and nrows < 20000:
+        ts = smp.rng.integers(0, cfg.seqlen, size=16)
+        hs = smp.rng.integers(0, cfg.group, size=16)
+        qrows = [S.gen_rows(cfg, "q", 0, int(t), int(t) + 1, int(h))[0] for t, h in zip(ts, hs)]
+        t1 = time.perf_counter()
+        for t, q in zip(ts, qrows):
+            sel = P.select_blocks_pooled(q, smp.kbar, kmax, kmin, int(t), cfg.block, cfg.topk, extra)
+            pos = O.key_positions(sel, int(t), cfg.block, cfg.seqlen)
+            O.attend_row(q, smp.K[pos], smp.V[pos], cfg.softmax_scale)
+            pairs += len(pos)
+        secs += time.perf_counter() - t1
+        nrows += 16
+    full_s = secs / nrows * cfg.batch * cfg.seqlen * cfg.hq + t_pools * cfg.batch * cfg.hkv
+    return {"cores": blas_threads(), "kind": "oracle", "extrapolated_full_layer_s": full_s,
+            "sample_tflops": 4.0 * cfg.head_dim * pairs / secs / 1e12,
+            "sample": (f"{nrows} random query rows of the {cfg.name} layer (fp64 pooled-gate oracle, "
+                       f"{secs:.1f} s) plus the three pools of one kv head ({t_pools:.1f} s), "
+                       f"extrapolated to the full layer")}
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -314,7 +344,7 @@ def backward_bench(cfg, steps, warmup):
                       "device_status": status}), flush=True)
 
 
-def pooled_gate_bench(cfg, extra, steps, warmup):
+def pooled_gate_bench(cfg, extra, steps, warmup, cpu_budget=None):
     """One JSON line: the layer with the gate variant that also routes the top
     `extra` blocks by max- and min-pooled keys (mean-pool, max/min-pool, the
     three-ranking gate, attention at width topk + 2 extra) beside the plain
@@ -364,13 +394,17 @@ def pooled_gate_bench(cfg, extra, steps, warmup):
     flops = routed_flops(cfg, routed)
     peaks, _ = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    cpu = None
+    if cpu_budget:
+        cpu = cpu_baseline_pooled(cfg, extra, cpu_budget)
+        cpu.update(value=flops / cpu["extrapolated_full_layer_s"] / 1e12, unit="TFLOP/s")
     print(json.dumps({"mode": "pooled_gate", "workload": cfg.name, "seqlen": cfg.seqlen, "topk": cfg.topk,
                       "extra": extra, "width": cfg.topk + 2 * extra, "ms_per_layer": ms_pooled,
                       "ms_per_layer_plain_gate": ms_plain, "stage_ms": stages,
                       "routed_pairs": routed, "routed_pairs_plain_gate": M.moba_rows_elems(plain.shape),
                       "tflops": flops / ms_pooled / 1e9, "frac_of_sustained_peak": flops / ms_pooled / 1e9 / peak,
                       "steps": steps, "warmup": warmup, "gpu_launches_per_step": pooled.launches,
-                      "device_status": list(pooled.device_status())}), flush=True)
+                      "device_status": list(pooled.device_status()), "cpu_baseline": cpu}), flush=True)
 
 
 def speedup_curve(seqlens, reps=2):
@@ -463,7 +497,8 @@ def main():
         speedup_curve([int(x) for x in args.curve_seqlens.split(",")])
         return
     if args.pooled_gate is not None:
-        pooled_gate_bench(S.get_config(args.config), args.pooled_gate, args.steps, args.warmup)
+        pooled_gate_bench(S.get_config(args.config), args.pooled_gate, args.steps, args.warmup,
+                          None if args.no_cpu_baseline else args.cpu_budget)
         return
     if args.backward:
         backward_bench(S.get_config(args.config), args.steps, args.warmup)

@@ -39,3 +39,11 @@ def test_routed_flops_of_the_pooled_gate_count_its_attended_keys():
     keys = sum(len(O.key_positions(sel, t, cfg.block, cfg.seqlen)) for (_, t, _), sel in sels.items())
     routed = sum(len(sel) - 1 for sel in sels.values())
     assert bench.routed_flops(cfg, routed) == 4.0 * cfg.head_dim * keys
+
+
+def test_pooled_cpu_baseline_runs_the_pooled_oracle_on_sampled_rows():
+    cfg = S.get_config("mqar").replace(batch=1, seqlen=2048, hq=4, hkv=2)
+    d = bench.cpu_baseline_pooled(cfg, 1, budget_s=0.5)
+    assert d["kind"] == "oracle" and d["cores"] >= 1
+    assert d["extrapolated_full_layer_s"] > 0 and d["sample_tflops"] > 0
+    assert "pooled-gate oracle" in d["sample"]
