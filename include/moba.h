@@ -104,7 +104,9 @@ MOBA_API int64_t moba_num_blocks(const moba_shape_t* shape);
  * tokens (for every batch entry at once) so that the per-block partial
  * results of one pass fit a bounded workspace.  query_chunk > 0 (a multiple
  * of 128) is used as given; 0 picks the largest power of two >= 128 whose
- * partials fit 8 GiB, capped at seqlen rounded up to 128. */
+ * partials fit 8 GiB, capped at seqlen rounded up to 128 (a partial takes
+ * 2 * head_dim + 4 bytes on the tensor-core path, bf16 with head_dim 128, and
+ * 4 * (head_dim + 1) bytes otherwise; 65536 tokens at 1M, 524288 at 10M). */
 MOBA_API int64_t moba_query_chunk(const moba_shape_t* shape);
 
 /* Number of passes: ceil(seqlen / C). */
@@ -394,10 +396,23 @@ MOBA_API moba_status_t moba_selftest_bounded_wait(int* status, moba_stream_t str
  *     capture on the device.
  *   - All calls on a device share the one array: calls that overlap on the GPU
  *     (different streams without ordering between them) race and give wrong
- *     results.  Order them on one stream or with events. */
+ *     results.  Order them on one stream or with events.
+ *   - The device status word (0, or MOBA_ERR_TIMEOUT when a bounded wait of the
+ *     tensor-core scoring kernel gave up and sel/offsets/rows are not valid) is
+ *     in the same array, at a fixed place; moba_gate_noalloc_status reads it. */
 MOBA_API moba_status_t moba_gate_topk_noalloc(const moba_shape_t* shape, const void* q,
                                               const float* meank, int32_t* sel, int32_t* offsets,
                                               int32_t* rows, moba_stream_t stream);
+
+/* Status word of the last moba_gate_topk_noalloc call on the current device:
+ * enqueues on `stream` a copy of the word into *status, HOST memory (pinned or
+ * pageable; with pageable memory the copy completes before this call returns).
+ * Read *status after `stream` has synchronised.  The word is cleared at the
+ * start of every moba_gate_topk_noalloc call, so order this call after the gate
+ * call it reports on (the same stream does that).  Allocates nothing.
+ * Returns MOBA_ERR_INVALID_ARG for a null pointer, MOBA_ERR_CUDA if the copy
+ * cannot be enqueued. */
+MOBA_API moba_status_t moba_gate_noalloc_status(int* status, moba_stream_t stream);
 
 #ifdef __cplusplus
 }

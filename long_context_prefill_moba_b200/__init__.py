@@ -34,7 +34,8 @@ __all__ = [
     "moba_num_blocks", "moba_query_chunk", "moba_num_chunks", "moba_meank_elems",
     "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems", "moba_gate_workspace_size",
     "moba_attn_workspace_size", "moba_block_meanpool", "moba_gate_topk", "moba_attn_fwd",
-    "moba_status_string", "moba_last_launch_count", "moba_gate_topk_noalloc", "MobaLayer", "moba_forward",
+    "moba_status_string", "moba_last_launch_count", "moba_gate_topk_noalloc",
+    "moba_gate_noalloc_status", "MobaLayer", "moba_forward",
     "moba_prefill_host_workspace_size", "moba_prefill_host", "MobaHostLayer",
     "moba_attn_bwd_workspace_size", "moba_attn_bwd", "moba_attention",
     "moba_pooled_wide_shape", "moba_block_maxminpool", "moba_gate_pooled", "moba_attn_fwd_pooled",
@@ -53,7 +54,8 @@ EXPORTED_SYMBOLS = [
     "moba_meank_elems", "moba_sel_elems", "moba_offsets_elems", "moba_rows_elems",
     "moba_gate_workspace_size", "moba_attn_workspace_size", "moba_block_meanpool",
     "moba_gate_topk", "moba_attn_fwd", "moba_status_string", "moba_last_cuda_error",
-    "moba_last_launch_count", "moba_gate_topk_noalloc", "moba_selftest_bounded_wait",
+    "moba_last_launch_count", "moba_gate_topk_noalloc", "moba_gate_noalloc_status",
+    "moba_selftest_bounded_wait",
     "moba_prefill_host_workspace_size", "moba_prefill_host", "moba_attn_bwd_workspace_size",
     "moba_attn_bwd", "moba_pooled_wide_shape", "moba_block_maxminpool", "moba_gate_pooled",
     "moba_attn_fwd_pooled", "moba_workspace_size", "moba_rows_capacity", "moba_check_index",
@@ -114,6 +116,8 @@ def load_library(path: str = LIB_PATH):
     L.moba_selftest_bounded_wait.restype = st
     L.moba_gate_topk_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp]
     L.moba_gate_topk_noalloc.restype = st
+    L.moba_gate_noalloc_status.argtypes = [vp, vp]
+    L.moba_gate_noalloc_status.restype = st
     L.moba_attn_bwd_workspace_size.argtypes = [P]
     L.moba_attn_bwd_workspace_size.restype = sz
     L.moba_attn_bwd.argtypes = [P] + [vp] * 13 + [sz, vp]
@@ -211,6 +215,16 @@ def moba_gate_topk_noalloc(shape, q, meank, sel, offsets, rows, stream=None):
     _check(lib().moba_gate_topk_noalloc(_s(shape), _ptr(q), _ptr(meank), _ptr(sel), _ptr(offsets),
                                         _ptr(rows), _stream(stream)),
            "moba_gate_topk_noalloc")
+
+
+def moba_gate_noalloc_status(stream=None) -> int:
+    """Device status word of the last moba_gate_topk_noalloc call on the current
+    device (0, or MOBA_ERR_TIMEOUT = 6); synchronises `stream`."""
+    word = ctypes.c_int(-1)
+    st = stream if stream is not None else torch.cuda.current_stream()
+    _check(lib().moba_gate_noalloc_status(ctypes.byref(word), _stream(st)), "moba_gate_noalloc_status")
+    st.synchronize()
+    return int(word.value)
 
 
 def moba_selftest_bounded_wait(status, stream=None):

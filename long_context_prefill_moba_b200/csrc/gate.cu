@@ -340,6 +340,7 @@ cudaError_t launch_gate_pass(const Dims& dm_all, int dtype, const void* q, const
 namespace {
 
 constexpr int kNoAllocMaxDevices = 64;
+constexpr int64_t kNoAllocStatusIndex = 2 * (int64_t)MOBA_GATE_NOALLOC_MAX_GROUPS;
 static __device__ __align__(256) int32_t g_gate_scratch[2 * MOBA_GATE_NOALLOC_MAX_GROUPS + 64];
 
 std::mutex g_scratch_mu;
@@ -374,8 +375,18 @@ cudaError_t launch_gate_noalloc(const Dims& dm, int dtype, const void* q, const 
   cudaError_t e = scratch_for_current_device(&scratch);
   if (e != cudaSuccess) return e;
   const int64_t L = (int64_t)dm.nchunks * dm.batch * dm.hkv * dm.n;
-  GateWs ws{scratch, scratch + L, scratch + 2 * L};   // counts, cursors, status; launch_gate clears them
+  // counts, cursors (launch_gate clears them) and the status word, which sits
+  // at a fixed index whatever the shape so that moba_gate_noalloc_status finds it
+  GateWs ws{scratch, scratch + L, scratch + kNoAllocStatusIndex};
   return launch_gate(dm, dtype, q, meank, sel, offsets, rows, ws, stream, launches);
+}
+
+cudaError_t gate_noalloc_status(int* host_status, cudaStream_t stream) {
+  int32_t* scratch = nullptr;
+  cudaError_t e = scratch_for_current_device(&scratch);
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyAsync(host_status, scratch + kNoAllocStatusIndex, sizeof(int), cudaMemcpyDeviceToHost,
+                         stream);
 }
 
 }  // namespace moba

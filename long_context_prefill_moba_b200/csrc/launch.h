@@ -47,6 +47,8 @@ cudaError_t launch_gate_pass(const Dims& dm, int dtype, const void* q, const flo
 cudaError_t launch_gate_noalloc(const Dims& dm, int dtype, const void* q, const float* meank,
                                 int32_t* sel, int32_t* offsets, int32_t* rows,
                                 cudaStream_t stream, int* launches);
+// copy of the allocation-free gate's device status word into host memory, on `stream`
+cudaError_t gate_noalloc_status(int* host_status, cudaStream_t stream);
 
 // exclusive prefix sum of in[0..L) plus `base` into out[0..L] (one CTA)
 cudaError_t launch_gate_scan(const int32_t* in, int32_t* out, int64_t L, int32_t base,

@@ -6,8 +6,10 @@
 //
 // HBM-bound: every key byte is read exactly once with 16-byte coalesced loads.
 // One CTA reduces one (batch, block, column slice): the warps of the CTA walk
-// disjoint rows of the block, keep fp32 sums in registers, and combine through
-// shared memory in a fixed order (deterministic result).
+// disjoint rows of the block, sum runs of four rows in fp32 and the runs in
+// fp64 registers, and combine through shared memory in a fixed order
+// (deterministic result); the mean is rounded to fp32 once, so the pooled keys
+// carry no error of a long fp32 running sum even for blocks of 40960 rows.
 #include "launch.h"
 
 namespace moba {
@@ -15,7 +17,7 @@ namespace moba {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 4;   // the fp32 run below adds exactly four rows
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) meanpool_kernel(const T* __restrict__ k,
@@ -34,9 +36,12 @@ __global__ void __launch_bounds__(kThreads) meanpool_kernel(const T* __restrict_
   const int t1 = min(N, t0 + B);
   const bool active = (rsub < rows_per_pass) && (cvec < vecs_per_row);
 
-  float acc[V];
+  // runs of kUnroll rows are summed in fp32 (pairwise), the runs in fp64: the
+  // pooled key is the fp32 rounding of a sum with ~1e-16 relative error, not
+  // of a long fp32 running sum
+  double acc[V];
 #pragma unroll
-  for (int i = 0; i < V; ++i) acc[i] = 0.f;
+  for (int i = 0; i < V; ++i) acc[i] = 0.0;
 
   if (active) {
     const T* base = k + ((size_t)b * N) * W + (size_t)cvec * V;
@@ -46,32 +51,30 @@ __global__ void __launch_bounds__(kThreads) meanpool_kernel(const T* __restrict_
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) Vec16<T>::load(base + (size_t)(t + u * rows_per_pass) * W, x[u]);
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-#pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] += x[u][i];
+      for (int i = 0; i < V; ++i) acc[i] += (double)((x[0][i] + x[1][i]) + (x[2][i] + x[3][i]));
     }
     for (; t < t1; t += rows_per_pass) {
       float x[V];
       Vec16<T>::load(base + (size_t)t * W, x);
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] += x[i];
+      for (int i = 0; i < V; ++i) acc[i] += (double)x[i];
     }
   }
 
   // combine the row-groups of the CTA: [rows_per_pass][cols_cta * V]
-  __shared__ float red[kThreads * V];
+  __shared__ double red[kThreads * V];
   if (rsub < rows_per_pass) {
 #pragma unroll
     for (int i = 0; i < V; ++i) red[rsub * cols_cta * V + (tid % cols_cta) * V + i] = acc[i];
   }
   __syncthreads();
-  const float inv = 1.f / (float)(t1 - t0);
+  const double len = (double)(t1 - t0);
   for (int e = tid; e < cols_cta * V; e += kThreads) {
     const int col = blockIdx.x * cols_cta * V + e;
     if (col >= W) continue;
-    float s = 0.f;
+    double s = 0.0;
     for (int r = 0; r < rows_per_pass; ++r) s += red[r * cols_cta * V + e];
-    meank[((size_t)b * n + j) * W + col] = s * inv;
+    meank[((size_t)b * n + j) * W + col] = (float)(s / len);
   }
 }
 

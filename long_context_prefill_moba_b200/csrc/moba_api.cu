@@ -24,7 +24,11 @@ int64_t chunk_of(const moba_shape_t* s) {
   if (s->query_chunk > 0) return s->query_chunk < cap ? s->query_chunk : cap;
   const int64_t KH = s->topk - 1;
   if (KH == 0) return cap;
-  const int64_t per_token = (int64_t)s->batch * s->hq * KH * (s->head_dim + 1) * 4;
+  // bytes of one partial result: bf16 output and fp32 log-sum-exp on the
+  // tensor-core path (bf16, head_dim 128), fp32 output and lse otherwise
+  const int64_t slot = s->dtype == MOBA_BF16 && s->head_dim == 128 ? 2 * s->head_dim + 4
+                                                                   : 4 * (s->head_dim + 1);
+  const int64_t per_token = (int64_t)s->batch * s->hq * KH * slot;
   int64_t c = 128;
   while (c * 2 <= cap && c * 2 * per_token <= kPartialBudget) c *= 2;
   return c < cap ? c : cap;
@@ -258,6 +262,12 @@ MOBA_API moba_status_t moba_gate_topk_noalloc(const moba_shape_t* s, const void*
   cudaError_t e = moba::launch_gate_noalloc(make_dims(s), s->dtype, q, meank, sel, offsets, rows,
                                             (cudaStream_t)stream, &launches);
   return finish(e, launches);
+}
+
+MOBA_API moba_status_t moba_gate_noalloc_status(int* status, moba_stream_t stream) {
+  g_last_launches = 0;
+  if (status == nullptr) return MOBA_ERR_INVALID_ARG;
+  return finish(moba::gate_noalloc_status(status, (cudaStream_t)stream), 0);
 }
 
 struct BwdLayout {

@@ -20,12 +20,14 @@ which lets the oracle rebuild exactly the rows it samples at 1M/10M tokens.
 Workload (the pages' shapes; the pages' own data are real text and an MQAR
 task that are not available, so these synthetic tensors stand in for them):
 
-    q[b,t,h,:] ~ N(0,1)
+    q[b,t,h,:] ~ q_std * N(0,1)                          (q_std = 1 unless stated)
     k[b,t,g,:] ~ N(0,1) + offset_std * o[b, t // B, g, :],   o ~ N(0,1)
     v[b,t,g,:] ~ N(0,1)
 
 The per-block key offset o makes the mean-pooled keys of different blocks
-differ, as the configs ask.  Values are drawn in fp32 and rounded once (RNE)
+differ, as the configs ask.  q_std and offset_std are powers of two, so the
+scalings are exact; q_std = 8 with offset_std = 4 gives gate scores q.meanK in
+the hundreds (std ~360), the magnitude of unscaled scores in trained models.  Values are drawn in fp32 and rounded once (RNE)
 to the config's dtype.
 """
 from __future__ import annotations
@@ -62,6 +64,13 @@ class MobaConfig:
     offset_std: float
     seed: int = 0
     scale: Optional[float] = None   # None -> 1/sqrt(d)
+    q_std: float = 1.0              # q = q_std * N(0,1); a power of two (exact)
+
+    def __post_init__(self):
+        for name in ("q_std", "offset_std"):
+            m, _ = math.frexp(getattr(self, name))
+            if m != 0.5:
+                raise ValueError(f"{name} must be a power of two (exact scaling)")
 
     @property
     def nblocks(self) -> int:
@@ -157,6 +166,8 @@ def gen_q(cfg: MobaConfig, device="cpu") -> torch.Tensor:
     """q as [batch, seqlen, hq, head_dim] in the config dtype."""
     n = cfg.batch * cfg.seqlen * cfg.hq * cfg.head_dim
     x = _flat_normals(0, n, cfg.seed, TENSOR_Q, device)
+    if cfg.q_std != 1.0:
+        x = x * cfg.q_std
     return _finish(x, cfg).view(cfg.batch, cfg.seqlen, cfg.hq, cfg.head_dim)
 
 
@@ -211,6 +222,8 @@ def gen_rows(cfg: MobaConfig, tensor: str, b: int, t0: int, t1: int, head: int,
     if tensor == "q":
         idx = (((b * cfg.seqlen + t) * cfg.hq + head) * d)[:, None] + e[None, :]
         x = _normals_at(idx.reshape(-1), cfg.seed, TENSOR_Q).view(t1 - t0, d)
+        if cfg.q_std != 1.0:
+            x = x * cfg.q_std
     elif tensor == "v":
         idx = (((b * cfg.seqlen + t) * cfg.hkv + head) * d)[:, None] + e[None, :]
         x = _normals_at(idx.reshape(-1), cfg.seed, TENSOR_V).view(t1 - t0, d)

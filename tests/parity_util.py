@@ -81,8 +81,14 @@ def check_index(layer, cfg, sel):
     assert np.array_equal(rows[got], r[exp])
 
 
-def full_parity(cfg, res):
-    """Whole-layer comparison with the dense-mask oracle (small configs)."""
+def out_err(got, exp, cfg, rel=0.0):
+    """max over elements of |got - exp| - rel * |exp| (<= out_tol(cfg) passes)."""
+    return float((np.abs(got - exp) - rel * np.abs(exp)).max())
+
+
+def full_parity(cfg, res, rel=0.0):
+    """Whole-layer comparison with the dense-mask oracle (small configs).
+    `rel` widens the output bound by rel * |expected| (see the large-score tests)."""
     q, k, v = S.gen_q(cfg), S.gen_k(cfg), S.gen_v(cfg)
     o_out, o_lse, o_sel, o_gap = O.moba_dense(q, k, v, cfg.block, cfg.topk, cfg.softmax_scale)
     layer = res["layer"]
@@ -107,7 +113,7 @@ def full_parity(cfg, res):
         pos = O.key_positions(used, t, cfg.block, cfg.seqlen)
         exp_out[b, t, h], exp_lse[b, h, t] = O.attend_row(qd[b, t, h], kd[b, pos, g], vd[b, pos, g],
                                                           cfg.softmax_scale)
-    err = np.abs(out - exp_out).max()
+    err = out_err(out, exp_out, cfg, rel)
     assert err <= out_tol(cfg), err
     if lse is not None:
         assert np.abs(lse - exp_lse).max() <= LSE_TOL[cfg.dtype]
@@ -115,11 +121,23 @@ def full_parity(cfg, res):
     return dict(max_err=float(err), n_gap_rows=len(differ[0]))
 
 
-def sampled_rows(cfg, n_random, seed=0):
-    """(b, h, t) rows: seeded random positions plus the boundary positions."""
+def sampled_rows(cfg, n_random, seed=0, chunk=0, max_pass_rows=16):
+    """(b, h, t) rows: seeded random positions plus fixed ones: the block and
+    sequence boundaries, a row of every regime with fewer earlier blocks than
+    slots (c < topk - 1) and the last token of each such block, and (with the
+    query pass length `chunk`) the first and last token of passes."""
     rng = np.random.default_rng(seed)
     B, N, k = cfg.block, cfg.seqlen, cfg.topk
     fixed_t = {0, B - 1, B, (k - 1) * B, N - 1, min(N - 1, (k - 2) * B + 7)}
+    for c in range(min(k - 1, cfg.nblocks)):
+        fixed_t |= {c * B + (37 * c + 5) % B, (c + 1) * B - 1}
+    if chunk > 0:
+        starts = list(range(chunk, N, chunk))
+        if len(starts) > max_pass_rows // 2:
+            pick = np.linspace(0, len(starts) - 1, max_pass_rows // 2).round().astype(int)
+            starts = [starts[i] for i in sorted(set(pick.tolist()))]
+        for p in starts:
+            fixed_t |= {p - 1, p}
     rows = []
     for i, t in enumerate(sorted(x for x in fixed_t if 0 <= x < N)):
         rows.append((int(i % cfg.batch), int((7 * i) % cfg.hq), int(t)))
@@ -128,8 +146,19 @@ def sampled_rows(cfg, n_random, seed=0):
     return rows
 
 
-def sampled_parity(cfg, res, rows):
-    """Row-by-row comparison with the gather oracle on regenerated rows."""
+def device_index_check(layer, exact=True):
+    """moba_check_index on the layer's own gate index (every row, on the
+    device); returns the status word (0 = valid)."""
+    import long_context_prefill_moba_b200 as M
+    status = torch.full((1,), -1, dtype=torch.int32, device=layer.device)
+    M.moba_check_index(layer.shape, exact, layer.sel, layer.offsets, layer.rows, status)
+    torch.cuda.synchronize()
+    return int(status.item())
+
+
+def sampled_parity(cfg, res, rows, rel=0.0):
+    """Row-by-row comparison with the gather oracle on regenerated rows (`rel` as
+    in full_parity)."""
     layer = res["layer"]
     sel_gpu = layer.sel_view()
     out_gpu = res["out"]
@@ -161,7 +190,7 @@ def sampled_parity(cfg, res, rows):
             Ksel = cpu(K[torch.from_numpy(pos)]).numpy()
             o, l = O.attend_row(qrow, Ksel, Vsel, cfg.softmax_scale)
             got = cpu(out_gpu[b, t, h]).numpy()
-            err = float(np.abs(got - o).max())
+            err = out_err(got, o, cfg, rel)
             worst = max(worst, err)
             assert err <= out_tol(cfg), (b, h, t, err)
             if lse_gpu is not None:

@@ -52,7 +52,9 @@ def test_sizes_of_the_1m_layer(L):
     assert M.moba_check_shape(s) == 0
     assert M.moba_num_blocks(s) == 256
     C = M.moba_query_chunk(s)
-    assert C % 128 == 0 and C * 32 * 11 * 129 * 4 <= 8 << 30
+    # the largest power of two whose bf16 partials (256 B + a 4-B lse each) fit 8 GiB
+    assert C % 128 == 0 and C * 32 * 11 * (128 * 2 + 4) <= 8 << 30 < 2 * C * 32 * 11 * (128 * 2 + 4)
+    assert C == 65536
     assert M.moba_num_chunks(s) == (1 << 20) // C
     assert M.moba_sel_elems(s) == (1 << 20) * 32 * 12
     assert M.moba_meank_elems(s) == 256 * 8 * 128
@@ -62,7 +64,9 @@ def test_sizes_of_the_1m_layer(L):
     assert M.moba_rows_elems(s) == exact
     assert M.moba_attn_workspace_size(s) >= C * 32 * 11 * (128 * 2 + 4)     # bf16 partials + fp32 lse
     f = shape(dtype="f32")
-    assert M.moba_attn_workspace_size(f) >= M.moba_query_chunk(f) * 32 * 11 * 129 * 4
+    Cf = M.moba_query_chunk(f)
+    assert M.moba_attn_workspace_size(f) >= Cf * 32 * 11 * 129 * 4
+    assert Cf * 32 * 11 * 129 * 4 <= 8 << 30 < 2 * Cf * 32 * 11 * 129 * 4
     assert M.moba_gate_workspace_size(s) >= 2 * 4 * M.moba_num_chunks(s) * 8 * 256
 
 

@@ -11,7 +11,8 @@ import torch
 
 import moba_synth as S
 import oracle as O
-from parity_util import (check_index, cpu, full_parity, run_gpu, sampled_parity, sampled_rows)
+from parity_util import (check_index, cpu, device_index_check, full_parity, run_gpu, sampled_parity,
+                         sampled_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -102,18 +103,55 @@ def test_exact_ties_pick_lower_block(cuda_device):
         assert s == [int(x) for x in sel[b, t, h] if x >= 0]
 
 
+def _chunk(res):
+    import long_context_prefill_moba_b200 as M
+    return M.moba_query_chunk(res["layer"].shape)
+
+
 def test_llama8b_128k_sampled(cuda_device):
     cfg = S.get_config("llama8b_128k")
     res = run_gpu(cfg)
-    worst = sampled_parity(cfg, res, sampled_rows(cfg, 40, seed=1))
+    worst = sampled_parity(cfg, res, sampled_rows(cfg, 64, seed=1, chunk=_chunk(res)))
+    assert device_index_check(res["layer"]) == 0
     print("llama8b_128k worst", worst)
+
+
+# Gate scores in the hundreds (q_std 8, key offsets of std 4: q.meanK has std
+# ~360 and reaches ~1800), the magnitude of unscaled scores in trained models:
+# the ranking must still be exact wherever the oracle's gap is >= 1e-3.
+LARGE = dict(q_std=8.0, offset_std=4.0)
+# The logits are large too (std ~34), so each row's softmax is nearly one-hot
+# and many outputs sit at an extreme value of v, |out| ~ 4: there one bf16 ulp
+# is 2^-5, so the output's own rounding (half an ulp, 0.0156) plus the bf16
+# partial results (2^-9 relative) can exceed the 2e-2 bound by themselves.  The
+# bound is widened by 2^-8 |expected|, the rounding of a bf16 output, for these
+# two tests only.
+LARGE_REL = 2.0 ** -8
+
+
+def test_mqar_large_scores_full(cuda_device):
+    cfg = S.get_config("mqar").replace(**LARGE)
+    res = run_gpu(cfg)
+    info = full_parity(cfg, res, rel=LARGE_REL)
+    print("mqar large scores", info)
+
+
+def test_llama8b_128k_large_scores_sampled(cuda_device):
+    cfg = S.get_config("llama8b_128k").replace(**LARGE)
+    res = run_gpu(cfg)
+    worst = sampled_parity(cfg, res, sampled_rows(cfg, 256, seed=5, chunk=_chunk(res)), rel=LARGE_REL)
+    assert device_index_check(res["layer"]) == 0
+    print("llama8b_128k large scores worst", worst)
 
 
 def test_1m_sampled(cuda_device):
     cfg = S.get_config("1m")
     res = run_gpu(cfg)
-    worst = sampled_parity(cfg, res, sampled_rows(cfg, 24, seed=2))
-    print("1m worst", worst)
+    rows = sampled_rows(cfg, 256, seed=2, chunk=_chunk(res))
+    worst = sampled_parity(cfg, res, rows)
+    # invariants and index consistency over all 33.5M rows, on the device
+    assert device_index_check(res["layer"]) == 0
+    print("1m worst", worst, "rows", len(rows))
     del res
     torch.cuda.empty_cache()
 
@@ -121,8 +159,10 @@ def test_1m_sampled(cuda_device):
 def test_10m_sampled(cuda_device):
     cfg = S.get_config("10m")
     res = run_gpu(cfg, with_lse=False)
-    worst = sampled_parity(cfg, res, sampled_rows(cfg, 6, seed=3))
-    print("10m worst", worst)
+    rows = sampled_rows(cfg, 64, seed=3, chunk=_chunk(res))
+    worst = sampled_parity(cfg, res, rows)
+    assert device_index_check(res["layer"]) == 0
+    print("10m worst", worst, "rows", len(rows))
     del res
     torch.cuda.empty_cache()
 

@@ -2,9 +2,10 @@
 partition, and the whole sharded layer on 2 and 4 gloo ranks on the CPU with
 the fp64 oracle standing in for the per-rank GPU layer (a test double passed
 as layer_factory).  K and V exist only on the source rank before the
-broadcast; the ranks' head-sharded outputs, gathered in rank order, must
+exchange (a scatter of disjoint kv heads, or a send to each kv head's leader
+and a broadcast in its subgroup); the ranks' head-sharded outputs, gathered in rank order, must
 equal the unsharded oracle layer exactly, and so must dq; dK and dV, summed
-onto the source rank by the backward's reduce, must equal the unsharded
+onto the source rank by the backward (gathered, or reduced per kv head), must equal the unsharded
 gradients up to the order of the sum."""
 import os
 import socket
@@ -70,7 +71,7 @@ def _inputs(b, N, hq, hkv, d):
             torch.randn(b, N, hkv, d, generator=g, dtype=torch.float64))
 
 
-def _worker(rank, world, port, shape, path):
+def _worker(rank, world, port, shape, path, src=0):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -78,11 +79,11 @@ def _worker(rank, world, port, shape, path):
         from long_context_prefill_moba_b200.sharded import ShardedMobaLayer
         b, N, hq, hkv, d, B, topk = shape
         q, k, v = _inputs(b, N, hq, hkv, d)
-        if rank != 0:                            # only the source rank holds K/V before the broadcast
-            k, v = torch.zeros_like(k), torch.zeros_like(v)
+        if rank != src:                          # only the source rank holds K/V before the exchange
+            k, v = None, None
         cfg = S.get_config("tiny").replace(batch=b, seqlen=N, hq=hq, hkv=hkv, head_dim=d, block=B, topk=topk,
                                            scale=0.3)
-        layer = ShardedMobaLayer.from_config(cfg, device="cpu", layer_factory=_OracleLayer)
+        layer = ShardedMobaLayer.from_config(cfg, device="cpu", src=src, layer_factory=_OracleLayer)
         q_loc = q[:, :, layer.h0:layer.h1].contiguous()
         out_loc = torch.empty_like(q_loc)
         lse_loc = torch.empty(b, layer.h1 - layer.h0, N, dtype=torch.float64)
@@ -99,7 +100,7 @@ def _worker(rank, world, port, shape, path):
         layer.backward(q_loc, out_loc, lse_loc, dout[:, :, layer.h0:layer.h1].contiguous(), dq_loc, dk, dv)
         dqs = [torch.empty_like(dq_loc) for _ in range(world)]
         dist.all_gather(dqs, dq_loc)
-        if rank == 0:
+        if rank == src:
             torch.save({"out": torch.cat(outs, 2), "lse": torch.cat(lses, 1), "dq": torch.cat(dqs, 2),
                         "dk": dk, "dv": dv, "dout": dout}, path)
     finally:
@@ -114,15 +115,17 @@ def _free_port():
     return port
 
 
-@pytest.mark.parametrize("shape,world", [
-    ((1, 70, 4, 2, 8, 16, 3), 2),     # kv heads split over the ranks
-    ((1, 70, 4, 1, 8, 16, 3), 2),     # one kv head: its query heads split (the 10M layer's case)
-    ((2, 45, 8, 2, 8, 10, 2), 4),     # two ranks per kv head, two batch entries
+@pytest.mark.parametrize("shape,world,src", [
+    ((1, 70, 4, 2, 8, 16, 3), 2, 0),     # kv heads split over the ranks (scatter / gather)
+    ((1, 40, 8, 4, 8, 10, 3), 4, 2),     # one kv head per rank, the source not rank 0
+    ((1, 70, 4, 1, 8, 16, 3), 2, 0),     # one kv head: its query heads split (the 10M layer's case)
+    ((2, 45, 8, 2, 8, 10, 2), 4, 0),     # two ranks per kv head, two batch entries
+    ((2, 45, 8, 2, 8, 10, 2), 4, 1),     # the same with a source that leads no subgroup
 ])
-def test_sharded_layer_equals_the_unsharded_layer(tmp_path, shape, world):
+def test_sharded_layer_equals_the_unsharded_layer(tmp_path, shape, world, src):
     import oracle as O
     path = str(tmp_path / "gathered.pt")
-    mp.start_processes(_worker, args=(world, _free_port(), shape, path), nprocs=world, join=True,
+    mp.start_processes(_worker, args=(world, _free_port(), shape, path, src), nprocs=world, join=True,
                        start_method="spawn")
     got = torch.load(path)
     b, N, hq, hkv, d, B, topk = shape

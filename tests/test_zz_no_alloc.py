@@ -7,7 +7,9 @@ has a variant whose counters live in a fixed device array inside the library.
 This test calls it through the C ABI twice in a row and checks each result
 against the regular moba_gate_topk on the same inputs: identical selections and
 offsets, and identical query rows in every group (their order inside a group is
-unspecified for both entry points).  The file is named to run last."""
+unspecified for both entry points).  After each call the gate's device status
+word, read back into host memory with moba_gate_noalloc_status, is 0 (no bounded
+wait gave up).  The file is named to run last."""
 import numpy as np
 import pytest
 import torch
@@ -51,6 +53,7 @@ def test_gate_noalloc_matches_gate(cuda_device, name, chunk):
         assert torch.equal(sel, ref_sel), call
         assert torch.equal(off, ref_off), call
         assert np.array_equal(_rows_by_group(off, rows), ref_rows), call
+        assert M.moba_gate_noalloc_status() == 0, call
 
 
 def test_gate_noalloc_rejects_oversized_shapes():
