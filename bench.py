@@ -411,8 +411,9 @@ def speedup_curve(seqlens, reps=2):
     """One JSON line per sequence length: the MoBA layer (mean-pool + gate +
     attention through the C ABI) against dense causal attention on the same
     q, k, v computed by torch's scaled_dot_product_attention (a library
-    FlashAttention-class kernel; cuDNN when available) and, where its index fits,
-    by this library itself with topk >= n (dense through the MoBA kernels)."""
+    FlashAttention-class kernel; cuDNN when available) and by this library's
+    own kernels (MoBA with a single block B = N and topk = 1, which is dense
+    causal attention)."""
     import long_context_prefill_moba_b200 as M
     from torch.nn.attention import SDPBackend, sdpa_kernel
     M.load_library()
@@ -437,14 +438,14 @@ def speedup_curve(seqlens, reps=2):
         layer = M.MobaLayer.from_config(cfg, dev)
         moba_ms = timed(lambda: layer.forward(q, k, v, out))
         del layer
-        dense_self = None
-        dcfg = cfg.replace(topk=min(16, cfg.nblocks + 1))
-        dshape = M.make_shape(dcfg.batch, dcfg.seqlen, dcfg.hq, dcfg.hkv, dcfg.head_dim, dcfg.block,
-                              dcfg.topk, dcfg.dtype)
-        if dcfg.topk > dcfg.nblocks and M.moba_check_shape(dshape) == 0:
-            dl = M.MobaLayer.from_config(dcfg, dev)
-            dense_self = timed(lambda: dl.forward(q, k, v, out))
-            del dl
+        # dense causal attention through this library's own kernels: MoBA with
+        # one block (B = N) and topk = 1 attends every earlier key; the
+        # current-block kernel runs it with its causal window starting at key 0,
+        # with no index and no partial results
+        dcfg = cfg.replace(block=N, topk=1)
+        dl = M.MobaLayer.from_config(dcfg, dev)
+        dense_self = timed(lambda: dl.forward(q, k, v, out))
+        del dl
         qt, kt, vt = (x.transpose(1, 2).contiguous() for x in (q, k, v))
         backend = None
         dense_ms = None
@@ -464,7 +465,9 @@ def speedup_curve(seqlens, reps=2):
             "dense_ms": dense_ms, "dense_backend": backend,
             "dense_tflops": None if dense_ms is None else dense_flops / dense_ms / 1e9,
             "speedup_vs_dense": None if dense_ms is None else dense_ms / moba_ms,
-            "dense_via_moba_kernels_ms": dense_self}), flush=True)
+            "dense_via_moba_kernels_ms": dense_self,
+            "dense_via_moba_kernels_tflops": dense_flops / dense_self / 1e9,
+            "speedup_vs_dense_via_moba_kernels": dense_self / moba_ms}), flush=True)
         del q, k, v, out, qt, kt, vt
         torch.cuda.empty_cache()
 

@@ -137,7 +137,9 @@ MOBA_DEV bool decode_tile(Tile& w, const int32_t* tile_start, const int32_t* off
     const int ntile = (t_end - t0 + kQT - 1) / kQT;
     const int pairs = (dm.G + 1) / 2;
     int idx = blockIdx.x;
-    const int tau = idx % ntile; idx /= ntile;
+    // the last token tiles of a block (or of the sequence, with one block) have
+    // the most keys: they start first, so the launch does not end on them
+    const int tau = ntile - 1 - idx % ntile; idx /= ntile;
     const int p = idx % pairs; idx /= pairs;
     w.g = idx % dm.hkv;
     w.b = idx / dm.hkv;

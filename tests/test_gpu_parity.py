@@ -144,6 +144,18 @@ def test_llama8b_128k_large_scores_sampled(cuda_device):
     print("llama8b_128k large scores worst", worst)
 
 
+def test_dense_causal_via_single_block_128k_sampled(cuda_device):
+    """MoBA with one block (B = N) and topk = 1 is dense causal attention: the
+    current-block kernel runs it with its causal window starting at key 0, with
+    no index and no partial results (the speed-up curve's dense baseline through
+    this library's own kernels)."""
+    cfg = S.get_config("llama8b_128k").replace(block=131072, topk=1)
+    res = run_gpu(cfg)
+    assert res["layer"].launches > 0
+    worst = sampled_parity(cfg, res, sampled_rows(cfg, 64, seed=9))
+    print("dense causal 128k worst", worst)
+
+
 def test_1m_sampled(cuda_device):
     cfg = S.get_config("1m")
     res = run_gpu(cfg)
