@@ -302,7 +302,8 @@ MOBA_API moba_status_t moba_block_maxminpool(const moba_shape_t* shape, const vo
                                              float* mink, moba_stream_t stream);
 
 /* The variant's gate.  Scores are fp32 dot products of q with the three pooled
- * keys.
+ * keys (bf16 with head_dim 128 and ceil((n - 1) / 32) <= W: tensor cores, one
+ * pass per ranking, each exact up to fp32 accumulation; otherwise CUDA cores).
  *   q, meank        as for moba_gate_topk                              (read)
  *   maxk, mink      outputs of moba_block_maxminpool                   (read)
  *   sel      [batch, seqlen, hq, W] int32 (written): the chosen earlier blocks

@@ -22,8 +22,11 @@
 // min(W - 1, c) slots per row, adds nothing for them.
 //
 // Launches of the gate: maxminpool (once per layer, beside the mean-pool),
-// pooled_select, the gate's prefix scan, pooled_scatter; of the attention:
-// pooled_fill before the two attention kernels of every pass.
+// the selection, the gate's prefix scan, pooled_scatter; of the attention:
+// pooled_fill before the two attention kernels of every pass.  The selection
+// runs on tensor cores (three passes of gate_select_tc, one per ranking; see
+// gate_tc.cu) for bf16 with head_dim 128 when a row's candidate mask fits its
+// sel entries, and on CUDA cores (pooled_select, below) otherwise.
 #include <float.h>
 
 #include "launch.h"
@@ -433,11 +436,17 @@ cudaError_t launch_gate_pooled(const Dims& dm, int dtype, int km, int extra, con
   cudaError_t e = cudaMemsetAsync(ws.counts, 0, sizeof(int32_t) * L * 2, stream);  // counts+cursors
   if (e != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(ws.status, 0, sizeof(int), stream)) != cudaSuccess) return e;
-  if (dtype == MOBA_BF16)
+  if (gate_tc_pooled_supported(dm, dtype)) {
+    // three tensor-core passes (mean, max, min rankings), the union in the last
+    e = launch_gate_select_tc_pooled(dm, km, extra, q, meank, maxk, mink, sel, ws.counts, ws.status, stream);
+    *launches += 3;
+  } else if (dtype == MOBA_BF16) {
     e = launch_pooled_select<__nv_bfloat16>(dm, km, extra, q, meank, maxk, mink, sel, ws.counts, stream);
-  else
+    ++*launches;
+  } else {
     e = launch_pooled_select<float>(dm, km, extra, q, meank, maxk, mink, sel, ws.counts, stream);
-  ++*launches;
+    ++*launches;
+  }
   if (e != cudaSuccess) return e;
   if ((e = launch_gate_scan(ws.counts, offsets, L, 0, stream)) != cudaSuccess) return e;
   ++*launches;

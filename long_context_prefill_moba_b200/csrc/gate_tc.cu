@@ -40,6 +40,17 @@
 //   warp 9     single-thread tcgen05.mma issuer
 // The MMA of one tile overlaps the selection of the other warpgroup's tile.
 // Requires bf16, head_dim 128 and at most 256 blocks.
+//
+// The gate variant with max- and min-pooled keys (the OpenReview discussion,
+// the authors' answer to W1 on block representations; reading G1: the union of
+// the top (k-1) blocks by the mean-pooled keys and the top `extra` by each of
+// the max- and min-pooled keys) runs the same kernel three times, once per
+// ranking, with the row's candidate mask carried between the passes in the
+// row's own sel entries (a W-wide row holds the ceil(c / 32) mask words): the
+// mean pass stores its mask, the max pass ORs into it, and the min pass ORs its
+// own, takes the union out of the mask in increasing order and counts it.  The
+// max and min pools are bf16 values (maxima of bf16 keys), so one bf16 term
+// represents them exactly.
 #include <cudaTypedefs.h>
 #include <float.h>
 
@@ -75,6 +86,15 @@ struct Ctl {
   int abort;
   int hist[kMaxBlocks];
 };
+
+// what one launch ranks and writes (see the file comment)
+struct GatePass {
+  const float* pool;   // pooled keys [b, n, hkv, d] fp32
+  int nterms;          // bf16 terms that represent them exactly: 3 (mean) or 1 (max, min)
+  int slots;           // blocks this ranking selects per row: topk - 1, or extra
+  int mode;            // kOutSel, kMaskStore, kMaskOr, kMaskUnion
+};
+constexpr int kOutSel = 0, kMaskStore = 1, kMaskOr = 2, kMaskUnion = 3;
 
 MOBA_DEV uint32_t bar(const uint64_t* b) { return smem_u32(b); }
 // AND of `v` over the 128 threads of selection warpgroup `wg` (named barrier 1 + wg)
@@ -152,8 +172,8 @@ MOBA_DEV uint32_t low_bits(int n) { return n <= 0 ? 0u : n >= 32 ? ~0u : ((1u <<
 
 template <int KB>
 __global__ void __launch_bounds__(kThreads, 1) gate_select_tc_kernel(
-    const __grid_constant__ CUtensorMap tmQ, const float* __restrict__ meank,
-    int32_t* __restrict__ sel, int32_t* __restrict__ counts, int* __restrict__ status, Dims dm) {
+    const __grid_constant__ CUtensorMap tmQ, const GatePass gp, int32_t* __restrict__ sel,
+    int32_t* __restrict__ counts, int* __restrict__ status, Dims dm) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ Ctl ctl;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -176,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_select_tc_kernel(
   const int ntiles = ttiles * nsub;                 // tile k: token tile k / nsub, heads (k % nsub) * GT..
   const int cmax_cta = (t_stop - 1) / dm.B;         // blocks [0, cmax_cta) may be candidates
   const int npad = max(16, (cmax_cta + 15) / 16 * 16);
-  const int KH = dm.topk - 1;
+  const int KH = gp.slots;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
@@ -203,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_select_tc_kernel(
     float x[8];
     if (jr < cmax_cta) {
       const float4* src = reinterpret_cast<const float4*>(
-          meank + (((size_t)b * dm.n + jr) * dm.hkv + g) * kD + c * 8);
+          gp.pool + (((size_t)b * dm.n + jr) * dm.hkv + g) * kD + c * 8);
       const float4 a = __ldg(src), e = __ldg(src + 1);
       x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = e.x; x[5] = e.y; x[6] = e.z; x[7] = e.w;
     } else {
@@ -226,10 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1) gate_select_tc_kernel(
     const uint32_t off = (c >> 3) * kKBHalf + sw128_off(jr, c & 7);
     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(khi + off), "r"(hi[0]), "r"(hi[1]),
                  "r"(hi[2]), "r"(hi[3]) : "memory");
-    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(kmid + off), "r"(mid[0]), "r"(mid[1]),
-                 "r"(mid[2]), "r"(mid[3]) : "memory");
-    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(klo + off), "r"(lo[0]), "r"(lo[1]),
-                 "r"(lo[2]), "r"(lo[3]) : "memory");
+    if (gp.nterms > 1) {
+      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(kmid + off), "r"(mid[0]), "r"(mid[1]),
+                   "r"(mid[2]), "r"(mid[3]) : "memory");
+      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(klo + off), "r"(lo[0]), "r"(lo[1]),
+                   "r"(lo[2]), "r"(lo[3]) : "memory");
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -342,20 +364,37 @@ __global__ void __launch_bounds__(kThreads, 1) gate_select_tc_kernel(
       mbar_arrive(bar(&ctl.s_free[wg]));
       if (valid) {
         int32_t* outp = sel + ((size_t)(b * dm.N + t) * dm.hq + h) * dm.topk;
-        int pos = 0;
+        if (gp.mode != kOutSel) {
+          // the candidate mask travels between the passes in the row's sel entries
+          const int nwc = (c + 31) >> 5;
+          if (gp.mode != kMaskStore) {
 #pragma unroll
-        for (int w = 0; w < kMaxBlocks / 32; ++w) {
-          uint32_t x = mw[w];
-          while (x) {
-            const int j = w * 32 + __ffs(x) - 1;
-            x &= x - 1;
-            outp[pos++] = j;
-            atomicAdd(&ctl.hist[j], 1);
+            for (int w = 0; w < kMaxBlocks / 32; ++w)
+              if (w < nwc) mw[w] |= (uint32_t)outp[w];
+          }
+          if (gp.mode != kMaskUnion) {
+#pragma unroll
+            for (int w = 0; w < kMaxBlocks / 32; ++w)
+              if (w < nwc) outp[w] = (int32_t)mw[w];
           }
         }
-        // pos == m unless a score was NaN (then the row keeps fewer blocks)
-        outp[pos] = c;
-        for (int i = pos + 1; i < dm.topk; ++i) outp[i] = -1;
+        if (gp.mode == kOutSel || gp.mode == kMaskUnion) {
+          int pos = 0;
+#pragma unroll
+          for (int w = 0; w < kMaxBlocks / 32; ++w) {
+            uint32_t x = mw[w];
+            while (x) {
+              const int j = w * 32 + __ffs(x) - 1;
+              x &= x - 1;
+              outp[pos++] = j;
+              atomicAdd(&ctl.hist[j], 1);
+            }
+          }
+          // pos is m for the plain gate unless a score was NaN (then the row
+          // keeps fewer blocks); for the union it is the size of the union
+          outp[pos] = c;
+          for (int i = pos + 1; i < dm.topk; ++i) outp[i] = -1;
+        }
       }
     }
   } else if (warp == 8) {
@@ -396,16 +435,16 @@ __global__ void __launch_bounds__(kThreads, 1) gate_select_tc_kernel(
           const uint32_t qa = base + kOffQ;
           const uint32_t d = tb + s * 256u;
           // smallest term first: the accumulator is still small while the
-          // low-order products are added
-#pragma unroll
-          for (int term = 0; term < kTerms; ++term) {
+          // low-order products are added (one term: hi only)
+          const int t0 = kTerms - gp.nterms;
+          for (int term = t0; term < kTerms; ++term) {
             const uint32_t kt = klo - term * kKB;   // lo, mid, hi
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t qo = (kk >> 2) * kHalfQ + (kk & 3) * 32;
               const uint32_t ko = (kk >> 2) * kKBHalf + (kk & 3) * 32;
               mma_ss(d, sdesc_sw128(qa + qo, 16, 1024), sdesc_sw128(kt + ko, 16, 1024), idesc,
-                     (term > 0 || kk > 0) ? 1u : 0u);
+                     (term > t0 || kk > 0) ? 1u : 0u);
             }
           }
         }
@@ -453,24 +492,18 @@ int gate_ctas(const Dims& dm) {
 }
 
 template <int KB>
-cudaError_t run_select(const CUtensorMap& mq, const Dims& dm, const float* meank, int32_t* sel,
+cudaError_t run_select(const CUtensorMap& mq, const Dims& dm, const GatePass& gp, int32_t* sel,
                        int32_t* counts, int* status, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(gate_select_tc_kernel<KB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  gate_select_tc_kernel<KB><<<gate_ctas(dm), kThreads, kSmemBytes, stream>>>(mq, meank, sel, counts,
+  gate_select_tc_kernel<KB><<<gate_ctas(dm), kThreads, kSmemBytes, stream>>>(mq, gp, sel, counts,
                                                                              status, dm);
   return cudaGetLastError();
 }
 
-}  // namespace
-
-bool gate_tc_supported(const Dims& dm, int dtype) {
-  return dtype == MOBA_BF16 && dm.d == kD && dm.n <= kMaxBlocks && encode_fn_gate() != nullptr;
-}
-
-cudaError_t launch_gate_select_tc(const Dims& dm, const void* q, const float* meank, int32_t* sel,
-                                  int32_t* counts, int* status, cudaStream_t stream) {
+cudaError_t run_pass(const Dims& dm, const void* q, const GatePass& gp, int32_t* sel, int32_t* counts,
+                     int* status, cudaStream_t stream) {
   // q viewed as [b * N][hq][d]: a box of 64 columns x GT heads x 128 / GT tokens
   // lands in shared memory as 128 rows of 128 bytes, token-major
   const int GT = (kRowsT % dm.G == 0) ? dm.G : 1;
@@ -484,10 +517,37 @@ cudaError_t launch_gate_select_tc(const Dims& dm, const void* q, const float* me
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const int kh = dm.topk - 1;   // list length of the sorting networks: 4, 8 or 16 >= topk - 1
-  return kh <= 4   ? run_select<4>(mq, dm, meank, sel, counts, status, stream)
-         : kh <= 8 ? run_select<8>(mq, dm, meank, sel, counts, status, stream)
-                   : run_select<16>(mq, dm, meank, sel, counts, status, stream);
+  // list length of the sorting networks: 4, 8 or 16 >= the ranking's slots
+  return gp.slots <= 4   ? run_select<4>(mq, dm, gp, sel, counts, status, stream)
+         : gp.slots <= 8 ? run_select<8>(mq, dm, gp, sel, counts, status, stream)
+                         : run_select<16>(mq, dm, gp, sel, counts, status, stream);
+}
+
+}  // namespace
+
+bool gate_tc_supported(const Dims& dm, int dtype) {
+  return dtype == MOBA_BF16 && dm.d == kD && dm.n <= kMaxBlocks && encode_fn_gate() != nullptr;
+}
+
+cudaError_t launch_gate_select_tc(const Dims& dm, const void* q, const float* meank, int32_t* sel,
+                                  int32_t* counts, int* status, cudaStream_t stream) {
+  return run_pass(dm, q, GatePass{meank, kTerms, dm.topk - 1, kOutSel}, sel, counts, status, stream);
+}
+
+bool gate_tc_pooled_supported(const Dims& dm, int dtype) {
+  // the candidate mask of a row (ceil(c / 32) words, c <= n - 1) must fit its W-wide sel row
+  return gate_tc_supported(dm, dtype) && (dm.n - 1 + 31) / 32 <= dm.topk;
+}
+
+cudaError_t launch_gate_select_tc_pooled(const Dims& dm, int km, int extra, const void* q,
+                                         const float* meank, const float* maxk, const float* mink,
+                                         int32_t* sel, int32_t* counts, int* status,
+                                         cudaStream_t stream) {
+  cudaError_t e = run_pass(dm, q, GatePass{meank, kTerms, km, kMaskStore}, sel, counts, status, stream);
+  if (e != cudaSuccess) return e;
+  e = run_pass(dm, q, GatePass{maxk, 1, extra, kMaskOr}, sel, counts, status, stream);
+  if (e != cudaSuccess) return e;
+  return run_pass(dm, q, GatePass{mink, 1, extra, kMaskUnion}, sel, counts, status, stream);
 }
 
 }  // namespace moba

@@ -31,6 +31,14 @@ struct GateWs {
 bool gate_tc_supported(const Dims& dm, int dtype);
 cudaError_t launch_gate_select_tc(const Dims& dm, const void* q, const float* meank, int32_t* sel,
                                   int32_t* counts, int* status, cudaStream_t stream);
+// the pooled variant's three rankings on tensor cores (mean, max, min), the
+// union written as the W-wide sel row (dm.topk = W) with its counts; requires
+// gate_tc_pooled_supported (the row's candidate mask must fit its sel entries)
+bool gate_tc_pooled_supported(const Dims& dm, int dtype);
+cudaError_t launch_gate_select_tc_pooled(const Dims& dm, int km, int extra, const void* q,
+                                         const float* meank, const float* maxk, const float* mink,
+                                         int32_t* sel, int32_t* counts, int* status,
+                                         cudaStream_t stream);
 cudaError_t launch_gate(const Dims& dm, int dtype, const void* q, const float* meank, int32_t* sel,
                         int32_t* offsets, int32_t* rows, GateWs ws, cudaStream_t stream,
                         int* launches);

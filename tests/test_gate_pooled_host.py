@@ -20,8 +20,13 @@ PROGRAM = r"""
 #include <set>
 #include <vector>
 
-// the two launchers gate_pooled.cu calls but this host program never runs
+// the launchers gate_pooled.cu calls but this host program never runs
 namespace moba {
+bool gate_tc_pooled_supported(const Dims&, int) { return false; }
+cudaError_t launch_gate_select_tc_pooled(const Dims&, int, int, const void*, const float*, const float*,
+                                         const float*, int32_t*, int32_t*, int*, cudaStream_t) {
+  return cudaErrorNotSupported;
+}
 cudaError_t launch_attn_passes(const Dims&, int, const void*, const void*, const void*, const int32_t*,
                                const int32_t*, const int32_t*, void*, float*, AttnWs, int, int,
                                cudaStream_t, int*) { return cudaErrorNotSupported; }
