@@ -54,32 +54,45 @@ MOBA_DEV void red_add_v4(float* dst, float a, float b, float c, float d) {
                : "memory");
 }
 
-// row r of q / dout (this warp's 64-column half) into the swizzled tile
-MOBA_DEV void load_half_row(uint32_t tile, int rho, int hf, const __nv_bfloat16* src, bool valid) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) cp_async16(tile + hf * kHalf + sw128_off(rho, c), src + hf * 64 + c * 8, valid);
-}
-
 // ============================================================================ dK, dV
 // Transposed products: S^T = K Q^T and dP^T = V dO^T put a key on every TMEM
 // lane, so P^T and dS^T stay in TMEM as bf16 and feed dV += P^T dO and
-// dK += dS^T Q as TS MMAs; shared memory holds K, V and two Q/dO row tiles,
-// and the next row tile loads while the current one computes.
-constexpr int kKvThreads = (kSoftmaxWarps + 1) * 32;
-constexpr uint32_t kKvOffK = 0, kKvOffV = kTile, kKvOffQ = 2 * kTile;   // Q/dO stage x at kKvOffQ + 2x kTile
-constexpr uint32_t kKvSmem = 6 * kTile + 1024;
+// dK += dS^T Q as TS MMAs.  Row tiles are 64 query rows:
+//   TMEM   two stages of S^T | dP^T (64 columns each) and the dV, dK
+//          accumulators (128 columns each): 512 columns;
+//   SMEM   the K and V tiles and four stages of q | dout row tiles (16 KB each).
+// The MMA issuer runs S^T, dP^T of row tile i and then dV, dK of tile i - 1,
+// so the elementwise warps work on one tile while the tensor core computes
+// the next; a gather warpgroup copies the rows of the tiles ahead (cp.async,
+// 16 bytes per request, three tiles in flight) with their lse, D and causal
+// limit.
+constexpr int kR = 64;                          // query rows per row tile
+constexpr int kStages = 4;                      // q | dout row-tile stages
+constexpr uint32_t kRHalf = kR * 128;           // 8 KB: one 64-column half of a row tile
+constexpr uint32_t kRTile = 2 * kRHalf;         // 16 KB: q (or dout) of a row tile
+constexpr uint32_t kRStage = 2 * kRTile;        // q then dout
+constexpr int kGatherWarps = 4;
+constexpr int kKvWarps = kSoftmaxWarps + kGatherWarps + 1;   // elementwise, gather, MMA issuer
+constexpr int kKvThreads = kKvWarps * 32;
+constexpr int kGatherWarp = kSoftmaxWarps;                    // first gather warp
+constexpr int kMmaWarp = kSoftmaxWarps + kGatherWarps;
+constexpr int kGatherLag = 2;          // row tiles in flight beyond the one published
+static_assert(kGatherLag <= kStages - 2, "the MMA must always find a published tile to proceed");
+constexpr uint32_t kKvOffK = 0, kKvOffV = kTile, kKvOffQ = 2 * kTile;   // stage x at kKvOffQ + x kRStage
+constexpr uint32_t kKvSmem = 2 * kTile + kStages * kRStage + 1024;
 
 constexpr int kMaxPassPrefix = 256;    // passes whose row-tile prefix is kept in shared memory
 
 struct KvCtl {
-  uint64_t kv_full, q_full[2], s_full, p_full, mm_done, drain;
+  uint64_t kv_full, q_full[kStages], q_free[kStages], s_full[2], p_full[2], mm_done, drain;
   int pass_tiles[kMaxPassPrefix + 1];   // routed row tiles of passes [0, p), this CTA's group
   int pass_r0[kMaxPassPrefix];          // first routed row of pass p's group
+  int pass_r1[kMaxPassPrefix];          // end of pass p's group
   uint32_t tmem_base;
   int abort;
-  float lse2[2][kT];   // per row of a stage: forward lse in log2 units (+inf: no row)
-  float dlt[2][kT];    // D = <dout, out>
-  int tmax[2][kT];     // last key the row may attend (its token for the block's own rows)
+  float lse2[kStages][kR];   // per row of a stage: forward lse in log2 units (+inf: no row)
+  float dlt[kStages][kR];    // D = <dout, out>
+  int tmax[kStages][kR];     // last key the row may attend (its token for the block's own rows)
 };
 
 // the query rows of row tile i of this key tile: the gate's groups of block j
@@ -87,7 +100,7 @@ struct KvCtl {
 struct RowTile {
   bool own;          // block j's own rows (causal) or routed rows
   int r0, cnt;       // routed: rows[r0 .. r0 + cnt)
-  int t0, h;         // own: tokens t0 .. t0 + 127 of head h
+  int t0, h;         // own: tokens t0 .. t0 + kR - 1 of head h
 };
 
 MOBA_DEV int kv_tiles(const int32_t* offsets, const Dims& dm, int b, int g, int j, int key0, int key_end,
@@ -96,27 +109,25 @@ MOBA_DEV int kv_tiles(const int32_t* offsets, const Dims& dm, int b, int g, int 
   hist_tiles = 0;
   for (int ch = 0; ch < dm.nchunks; ++ch) {
     const int64_t gi = ch * ngroups + ((int64_t)b * dm.hkv + g) * dm.n + j;
-    hist_tiles += (offsets[gi + 1] - offsets[gi] + kT - 1) / kT;
+    hist_tiles += (offsets[gi + 1] - offsets[gi] + kR - 1) / kR;
   }
-  return hist_tiles + (key_end - key0 + kT - 1) / kT * dm.G;
+  return hist_tiles + (key_end - key0 + kR - 1) / kR * dm.G;
 }
 
 MOBA_DEV RowTile kv_row_tile(int i, int hist_tiles, const int32_t* offsets, const Dims& dm, int b, int g, int j,
-                             int key0, const int* pass_tiles, const int* pass_r0) {
+                             int key0, const int* pass_tiles, const int* pass_r0, const int* pass_r1) {
   RowTile rt{};
   if (i < hist_tiles && pass_tiles != nullptr) {
-    // the pass holding tile i: largest p with pass_tiles[p] <= i
+    // the pass holding tile i: largest p with pass_tiles[p] <= i (all in shared memory)
     int lo = 0, hi = dm.nchunks - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (pass_tiles[mid] <= i) lo = mid; else hi = mid - 1;
     }
     const int left = i - pass_tiles[lo];
-    const int64_t ngroups = (int64_t)dm.batch * dm.hkv * dm.n;
-    const int64_t gi = lo * ngroups + ((int64_t)b * dm.hkv + g) * dm.n + j;
     rt.own = false;
-    rt.r0 = pass_r0[lo] + left * kT;
-    rt.cnt = min(kT, offsets[gi + 1] - rt.r0);
+    rt.r0 = pass_r0[lo] + left * kR;
+    rt.cnt = min(kR, pass_r1[lo] - rt.r0);
     return rt;
   }
   if (i < hist_tiles) {
@@ -125,11 +136,11 @@ MOBA_DEV RowTile kv_row_tile(int i, int hist_tiles, const int32_t* offsets, cons
     for (int ch = 0; ch < dm.nchunks; ++ch) {
       const int64_t gi = ch * ngroups + ((int64_t)b * dm.hkv + g) * dm.n + j;
       const int r0 = offsets[gi], n = offsets[gi + 1] - r0;
-      const int nt = (n + kT - 1) / kT;
+      const int nt = (n + kR - 1) / kR;
       if (left < nt) {
         rt.own = false;
-        rt.r0 = r0 + left * kT;
-        rt.cnt = min(kT, n - left * kT);
+        rt.r0 = r0 + left * kR;
+        rt.cnt = min(kR, n - left * kR);
         return rt;
       }
       left -= nt;
@@ -137,16 +148,16 @@ MOBA_DEV RowTile kv_row_tile(int i, int hist_tiles, const int32_t* offsets, cons
   }
   const int k = i - hist_tiles;
   rt.own = true;
-  rt.t0 = key0 + (k / dm.G) * kT;
+  rt.t0 = key0 + (k / dm.G) * kR;
   rt.h = g * dm.G + k % dm.G;
   return rt;
 }
 
-// OR of `v` over the 256 softmax threads (named barrier 1); also a barrier
-MOBA_DEV bool softmax_any(bool v) {
+// AND of `v` over the 256 elementwise threads (named barrier 1)
+MOBA_DEV bool elementwise_all(bool v) {
   uint32_t r;
   asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, 256, p;\n"
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 256, p;\n"
       " selp.u32 %0, 1, 0, q;\n}\n"
       : "=r"(r)
       : "r"((uint32_t)v)
@@ -173,7 +184,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
   const int key_end = min(dm.N, (j + 1) * dm.B);
   if (b >= dm.batch || key0 >= key_end) return;
   int hist_tiles;
-  const int ntiles = kv_tiles(offsets, dm, b, g, j, key0, key_end, hist_tiles);
+  const int ntiles = kv_tiles(offsets, dm, b, g, j, key0, key_end, hist_tiles);   // >= G: own rows
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool prefix = dm.nchunks <= kMaxPassPrefix;
@@ -184,159 +195,81 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
       const int64_t gi = ch * ngroups + ((int64_t)b * dm.hkv + g) * dm.n + j;
       ctl.pass_tiles[ch] = acc;
       ctl.pass_r0[ch] = offsets[gi];
-      acc += (offsets[gi + 1] - offsets[gi] + kT - 1) / kT;
+      ctl.pass_r1[ch] = offsets[gi + 1];
+      acc += (offsets[gi + 1] - offsets[gi] + kR - 1) / kR;
     }
     ctl.pass_tiles[dm.nchunks] = acc;
   }
-  const int* pt = prefix ? ctl.pass_tiles : nullptr;
-  const int* pr = prefix ? ctl.pass_r0 : nullptr;
   if (tid == 0) {
-    mbar_init(bar(&ctl.kv_full), kSoftmaxWarps);
-    mbar_init(bar(&ctl.q_full[0]), kSoftmaxWarps);
-    mbar_init(bar(&ctl.q_full[1]), kSoftmaxWarps);
-    mbar_init(bar(&ctl.s_full), 1);
-    mbar_init(bar(&ctl.p_full), kSoftmaxWarps);
+    mbar_init(bar(&ctl.kv_full), kGatherWarps);
+    for (int x = 0; x < kStages; ++x) {
+      mbar_init(bar(&ctl.q_full[x]), kGatherWarps);
+      mbar_init(bar(&ctl.q_free[x]), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(&ctl.s_full[x]), 1);
+      mbar_init(bar(&ctl.p_full[x]), kSoftmaxWarps);
+    }
     mbar_init(bar(&ctl.mm_done), 1);
     mbar_init(bar(&ctl.drain), 1);
     ctl.abort = 0;
     fence_mbar_init();
   }
-  if (warp == kSoftmaxWarps) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(&ctl.tmem_base), 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const int* pt = prefix ? ctl.pass_tiles : nullptr;
+  const int* pr = prefix ? ctl.pass_r0 : nullptr;
+  const int* pe = prefix ? ctl.pass_r1 : nullptr;
   const uint32_t tb = ctl.tmem_base;
   volatile int* abort_flag = &ctl.abort;
 
   if (warp < kSoftmaxWarps) {
+    // ------------------------------------------------------------ elementwise
     const int qd = warp & 3, hf = warp >> 2;
     const int rho = qd * 32 + lane;           // TMEM lane: a key of S^T, dP^T, dK, dV
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const float sl2 = dm.scale_log2;
     const int u = key0 + rho;                  // this thread's key
     const bool key_ok = u < key_end;
-    {
-      const size_t kr = ((size_t)b * dm.N + (key_ok ? u : 0)) * dm.hkv + g;
-      load_half_row(base + kKvOffK, rho, hf, k + kr * kD, key_ok);
-      load_half_row(base + kKvOffV, rho, hf, v + kr * kD, key_ok);
-      cp_async_commit();
-    }
-    // the metadata of row tile i for this thread's row (its gathered row id,
-    // lse, D and causal limit) is read one tile ahead, so a tile's copies can
-    // start as soon as its stage is free
-    struct Meta {
-      int r, tmax;
-      float lse2, dlt;
-      bool valid;
-    };
-    auto meta_of = [&](int i) -> Meta {
-      Meta m{0, 0x7fffffff, INFINITY, 0.f, false};
-      if (i >= ntiles) return m;
-      const RowTile rt = kv_row_tile(i, hist_tiles, offsets, dm, b, g, j, key0, pt, pr);
-      int t, h;
-      if (rt.own) {
-        t = rt.t0 + rho;
-        h = rt.h;
-        m.valid = t < key_end;
-        m.r = (b * dm.N + t) * dm.hq + h;
-        m.tmax = t;
-      } else {
-        m.valid = rho < rt.cnt;
-        m.r = m.valid ? rows[rt.r0 + rho] : 0;
-        h = m.r % dm.hq;
-        t = (m.r / dm.hq) % dm.N;
-      }
-      if (m.valid) {
-        m.lse2 = lse[((size_t)b * dm.hq + h) * dm.N + t] * kLog2e;
-        m.dlt = delta[m.r];
-      } else {
-        m.r = 0;
-      }
-      return m;
-    };
-    // row tile i into stage i & 1: this thread loads half of its row's q and
-    // dout; the hf = 0 warp writes the row's scalars
-    auto load_tile = [&](int i, const Meta& m) {
-      const int x = i & 1;
-      const uint32_t sq = base + kKvOffQ + 2u * x * kTile;
-      load_half_row(sq, rho, hf, q + (size_t)m.r * kD, m.valid);
-      load_half_row(sq + kTile, rho, hf, dout + (size_t)m.r * kD, m.valid);
-      cp_async_commit();
-      if (hf == 0) {
-        ctl.lse2[x][rho] = m.lse2;
-        ctl.dlt[x][rho] = m.dlt;
-        ctl.tmax[x][rho] = m.tmax;
-      }
-    };
-    load_tile(0, meta_of(0));
-    Meta next = meta_of(1);
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    bool fail = softmax_any(false);   // scalars of stage 0 visible to every softmax thread
-    __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(bar(&ctl.kv_full));
-      mbar_arrive(bar(&ctl.q_full[0]));
-    }
-    for (int i = 0; i < ntiles; ++i) {
-      const int x = i & 1;
-      const bool more = i + 1 < ntiles;
-      if (more) {
-        // stage x ^ 1 held row tile i - 1: free once its MMAs completed
-        if (i >= 1 && !fail)
-          fail = !__all_sync(0xffffffffu, mbar_wait(bar(&ctl.mm_done), (i - 1) & 1, abort_flag));
-        if (!fail) {
-          load_tile(i + 1, next);
-          next = meta_of(i + 2);
-        }
-      }
-      if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(bar(&ctl.s_full), i & 1, abort_flag));
-      if (!fail) {
-        tc_fence_after();
-        uint32_t sr[64], dr[64];
-        tmem_ld32(tb + 64u * hf + lane_off, sr);
-        tmem_ld32(tb + 64u * hf + 32 + lane_off, sr + 32);
-        tmem_ld32(tb + 128u + 64u * hf + lane_off, dr);
-        tmem_ld32(tb + 128u + 64u * hf + 32 + lane_off, dr + 32);
-        tmem_wait_ld();
-        uint32_t pp[32], ps[32];
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int x = i & 1, st = i % kStages;
+      ok = elementwise_all(mbar_wait(bar(&ctl.s_full[x]), (i >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      // this warp's 32 rows of the tile: columns [32 hf, 32 hf + 32) of S^T_x and dP^T_x
+      const uint32_t cS = 64u * x + 32u * hf, cP = 128u + 64u * x + 32u * hf;
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tb + cS + lane_off, sr);
+      tmem_ld32(tb + cP + lane_off, dr);
+      tmem_wait_ld();
+      uint32_t pp[16], ps[16];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int ra = 64 * hf + 2 * c, rb = ra + 1;   // rows of this column pair
-          float p0 = ex2_approx(__uint_as_float(sr[2 * c]) * sl2 - ctl.lse2[x][ra]);
-          float p1 = ex2_approx(__uint_as_float(sr[2 * c + 1]) * sl2 - ctl.lse2[x][rb]);
-          p0 = (key_ok && u <= ctl.tmax[x][ra]) ? p0 : 0.f;
-          p1 = (key_ok && u <= ctl.tmax[x][rb]) ? p1 : 0.f;
-          pp[c] = pack_bf16x2(p0, p1);
-          ps[c] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * c]) - ctl.dlt[x][ra]),
-                              p1 * (__uint_as_float(dr[2 * c + 1]) - ctl.dlt[x][rb]));
-        }
-        // P^T and dS^T over this warp's own S^T / dP^T columns [64 hf, 64 hf + 32): already read
-        tmem_st32(tb + 64u * hf + lane_off, pp);
-        tmem_st32(tb + 128u + 64u * hf + lane_off, ps);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(&ctl.p_full));
+      for (int c = 0; c < 16; ++c) {
+        const int ra = 32 * hf + 2 * c, rb = ra + 1;   // rows of this column pair
+        float p0 = ex2_approx(__uint_as_float(sr[2 * c]) * sl2 - ctl.lse2[st][ra]);
+        float p1 = ex2_approx(__uint_as_float(sr[2 * c + 1]) * sl2 - ctl.lse2[st][rb]);
+        p0 = (key_ok && u <= ctl.tmax[st][ra]) ? p0 : 0.f;
+        p1 = (key_ok && u <= ctl.tmax[st][rb]) ? p1 : 0.f;
+        pp[c] = pack_bf16x2(p0, p1);
+        ps[c] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * c]) - ctl.dlt[st][ra]),
+                            p1 * (__uint_as_float(dr[2 * c + 1]) - ctl.dlt[st][rb]));
       }
-      if (more) {
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-      }
-      // one barrier per tile: the next stage's scalars are visible, and every
-      // softmax warp learns of a failure in any of them
-      if (softmax_any(fail)) {
-        fail = true;
-        break;
-      }
+      // P^T and dS^T over the first half of this warp's own columns (already read)
+      tmem_st16(tb + cS + lane_off, pp);
+      tmem_st16(tb + cP + lane_off, ps);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
-      if (more && lane == 0) mbar_arrive(bar(&ctl.q_full[x ^ 1]));
+      if (lane == 0) mbar_arrive(bar(&ctl.p_full[x]));
     }
-    if (!fail) fail = !__all_sync(0xffffffffu, mbar_wait(bar(&ctl.mm_done), (ntiles - 1) & 1, abort_flag));
-    if (!fail) {
+    if (ok) ok = elementwise_all(mbar_wait(bar(&ctl.mm_done), 0, abort_flag));
+    if (ok) {
       // dK, dV rows (lanes = keys) of this warp's 64 columns
       tc_fence_after();
       const float scale = sl2 / kLog2e;
@@ -366,49 +299,174 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
         }
       }
     }
+  } else if (warp < kMmaWarp) {
+    // ------------------------------------------------------------ gather
+    const int gw = warp - kGatherWarp;
+    {
+      // K and V of the tile: this warp's 32 keys, two per copy instruction
+      // (lanes 0-15 the 16 chunks of one key's row, lanes 16-31 the next's)
+      const int cc = lane & 15;
+#pragma unroll
+      for (int k2 = 0; k2 < 16; ++k2) {
+        const int key = 32 * gw + 2 * k2 + (lane >> 4);
+        const bool kok = key0 + key < key_end;
+        const size_t kr = ((size_t)b * dm.N + (kok ? key0 + key : 0)) * dm.hkv + g;
+        const uint32_t off = (cc >> 3) * kHalf + sw128_off(key, cc & 7);
+        cp_async16(base + kKvOffK + off, k + kr * kD + cc * 8, kok);
+        cp_async16(base + kKvOffV + off, v + kr * kD + cc * 8, kok);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(&ctl.kv_full));
+    }
+    // the warp's 16 rows of a row tile: lane l (and l + 16) holds row
+    // 16 gw + (l & 15) with its id, lse, D and causal limit.  The dependent
+    // loads are pipelined over the tiles: the row id of tile i + 2 (a read of
+    // `rows`), then lse and D of tile i + 1 (reads at that id), so that tile
+    // i's copies start without waiting on either.  Each copy instruction reads
+    // two whole 256-byte rows (lanes 0-15 one row's 16 chunks, 16-31 the next).
+    const int rr = 16 * gw + (lane & 15), cc = lane & 15;
+    struct RowOf {
+      int r, t, h, tmax;
+      bool valid;
+    };
+    struct Scal {
+      float lse2, dlt;
+    };
+    auto row_of = [&](int i) -> RowOf {
+      RowOf m{0, 0, 0, 0x7fffffff, false};
+      if (i >= ntiles) return m;
+      const RowTile rt = kv_row_tile(i, hist_tiles, offsets, dm, b, g, j, key0, pt, pr, pe);
+      if (rt.own) {
+        m.t = rt.t0 + rr;
+        m.h = rt.h;
+        m.valid = m.t < key_end;
+        m.r = m.valid ? (b * dm.N + m.t) * dm.hq + m.h : 0;
+        m.tmax = m.t;
+      } else {
+        m.valid = rr < rt.cnt;
+        m.r = m.valid ? rows[rt.r0 + rr] : 0;   // t and h follow from r once it has arrived
+        m.t = -1;
+      }
+      return m;
+    };
+    auto scal_of = [&](RowOf& m) -> Scal {
+      Scal c{INFINITY, 0.f};
+      if (!m.valid) return c;
+      if (m.t < 0) {
+        m.h = m.r % dm.hq;
+        m.t = (m.r / dm.hq) % dm.N;
+      }
+      c.lse2 = lse[((size_t)b * dm.hq + m.h) * dm.N + m.t] * kLog2e;
+      c.dlt = delta[m.r];
+      return c;
+    };
+    RowOf r0 = row_of(0), r1 = row_of(1);
+    Scal c0 = scal_of(r0);
+    bool ok = true;
+    int published = 0;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int st = i % kStages;
+      // stage st held row tile i - kStages: free once its dV, dK MMAs completed
+      if (i >= kStages) ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.q_free[st]), ((i / kStages) - 1) & 1,
+                                                                abort_flag));
+      if (!ok) break;
+      const RowOf r2 = row_of(i + 2);
+      const Scal c1 = scal_of(r1);
+      const uint32_t sq = base + kKvOffQ + (uint32_t)st * kRStage, sdo = sq + kRTile;
+#pragma unroll
+      for (int k2 = 0; k2 < 8; ++k2) {
+        const int rl = 2 * k2 + (lane >> 4);
+        const int rs = __shfl_sync(0xffffffffu, r0.r, rl);
+        const bool vs = __shfl_sync(0xffffffffu, r0.valid, rl);
+        const uint32_t off = (cc >> 3) * kRHalf + sw128_off(16 * gw + rl, cc & 7);
+        cp_async16(sq + off, q + (size_t)rs * kD + cc * 8, vs);
+        cp_async16(sdo + off, dout + (size_t)rs * kD + cc * 8, vs);
+      }
+      if (lane < 16) {
+        ctl.lse2[st][rr] = c0.lse2;
+        ctl.dlt[st][rr] = c0.dlt;
+        ctl.tmax[st][rr] = r0.tmax;
+      }
+      cp_async_commit();
+      // row tile i - kGatherLag has landed once at most kGatherLag groups are pending
+      if (i >= kGatherLag) {
+        cp_async_wait<kGatherLag>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(&ctl.q_full[(i - kGatherLag) % kStages]));
+        published = i - kGatherLag + 1;
+      }
+      r0 = r1;
+      c0 = c1;
+      r1 = r2;
+    }
+    cp_async_wait<0>();
+    if (ok) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      for (int i = published; i < ntiles; ++i)
+        if (lane == 0) mbar_arrive(bar(&ctl.q_full[i % kStages]));
+    }
   } else if (lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t idS = idesc_bf16(128, kT, false);     // A, B K-major
-    const uint32_t idG = idesc_bf16(128, kD, true);      // A from TMEM, B MN-major
+    const uint32_t idS = idesc_bf16(128, kR, false);     // A (K, V tile), B (q, dout rows) K-major
+    const uint32_t idG = idesc_bf16(128, kD, true);      // A from TMEM, B (q, dout rows) MN-major
     const uint32_t hi = sdesc_hi(1024);
     const uint32_t loK = sdesc_lo(base + kKvOffK, 16), loV = sdesc_lo(base + kKvOffV, 16);
-    bool ok = mbar_wait(bar(&ctl.kv_full), 0, abort_flag);
-    for (int i = 0; i < ntiles && ok; ++i) {
+    // dV += P^T dO and dK += dS^T Q of row tile i (TMEM stage i & 1, smem stage i % kStages):
+    // K runs over its 64 rows (rows 0-31 in columns 0-15 of P^T / dS^T, rows 32-63 in 32-47)
+    auto issue_grad = [&](int i) {
       const int x = i & 1;
-      const uint32_t sq = base + kKvOffQ + 2u * x * kTile, sdo = sq + kTile;
-      const uint32_t loQ = sdesc_lo(sq, 16), loDO = sdesc_lo(sdo, 16);
-      const uint32_t mnQ = sdesc_lo(sq, kHalf), mnDO = sdesc_lo(sdo, kHalf);
-      if (!(ok = mbar_wait(bar(&ctl.q_full[x]), (i >> 1) & 1, abort_flag))) break;
-      tc_fence_after();
+      const uint32_t sq = base + kKvOffQ + (uint32_t)(i % kStages) * kRStage, sdo = sq + kRTile;
+      const uint32_t mnQ = sdesc_lo(sq, kRHalf), mnDO = sdesc_lo(sdo, kRHalf);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-        mma_ss(tb, sdesc_join(loK + off, hi), sdesc_join(loQ + off, hi), idS, kk > 0);
-      }
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-        mma_ss(tb + 128u, sdesc_join(loV + off, hi), sdesc_join(loDO + off, hi), idS, kk > 0);
-      }
-      mma_commit(bar(&ctl.s_full));
-      if (!(ok = mbar_wait(bar(&ctl.p_full), i & 1, abort_flag))) break;
-      tc_fence_after();
-      // dV += P^T dO, dK += dS^T Q: K runs over the 128 rows (rows 0-63 in
-      // columns 0-31 of P^T / dS^T, rows 64-127 in columns 64-95)
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t a = kk < 4 ? kk * 8u : 64u + (kk - 4) * 8u;
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t a = 64u * x + (kk < 2 ? kk * 8u : 32u + (kk - 2) * 8u);
         mma_ts(tb + 256u, tb + a, sdesc_join(mnDO + ((kk * 2048) >> 4), hi), idG, (i > 0 || kk > 0) ? 1u : 0u);
       }
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t a = kk < 4 ? kk * 8u : 64u + (kk - 4) * 8u;
-        mma_ts(tb + 384u, tb + 128u + a, sdesc_join(mnQ + ((kk * 2048) >> 4), hi), idG,
-               (i > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t a = 128u + 64u * x + (kk < 2 ? kk * 8u : 32u + (kk - 2) * 8u);
+        mma_ts(tb + 384u, tb + a, sdesc_join(mnQ + ((kk * 2048) >> 4), hi), idG, (i > 0 || kk > 0) ? 1u : 0u);
       }
-      mma_commit(bar(&ctl.mm_done));
+      mma_commit(bar(&ctl.q_free[i % kStages]));
+    };
+    bool ok = mbar_wait(bar(&ctl.kv_full), 0, abort_flag);
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int x = i & 1, st = i % kStages;
+      const uint32_t sq = base + kKvOffQ + (uint32_t)st * kRStage, sdo = sq + kRTile;
+      const uint32_t loQ = sdesc_lo(sq, 16), loDO = sdesc_lo(sdo, 16);
+      if (!(ok = mbar_wait(bar(&ctl.q_full[st]), (i / kStages) & 1, abort_flag))) break;
+      tc_fence_after();
+      // S^T_x, dP^T_x: stage x last held tile i - 2, whose dV, dK were issued before
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t offA = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+        const uint32_t offB = ((kk >> 2) * kRHalf + (kk & 3) * 32) >> 4;
+        mma_ss(tb + 64u * x, sdesc_join(loK + offA, hi), sdesc_join(loQ + offB, hi), idS, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t offA = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+        const uint32_t offB = ((kk >> 2) * kRHalf + (kk & 3) * 32) >> 4;
+        mma_ss(tb + 128u + 64u * x, sdesc_join(loV + offA, hi), sdesc_join(loDO + offB, hi), idS, kk > 0);
+      }
+      mma_commit(bar(&ctl.s_full[x]));
+      if (i >= 1) {
+        if (!(ok = mbar_wait(bar(&ctl.p_full[(i - 1) & 1]), ((i - 1) >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_grad(i - 1);
+      }
     }
-    if (!ok) {
+    if (ok) ok = mbar_wait(bar(&ctl.p_full[(ntiles - 1) & 1]), ((ntiles - 1) >> 1) & 1, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      issue_grad(ntiles - 1);
+      mma_commit(bar(&ctl.mm_done));
+    } else {
       int never = 0;
       mma_commit(bar(&ctl.drain));
       mbar_wait(bar(&ctl.drain), 0, &never);
@@ -418,7 +476,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kSoftmaxWarps) tmem_dealloc(tb, 512);
+  if (warp == kMmaWarp) tmem_dealloc(tb, 512);
   if (tid == 0 && ctl.abort) atomicExch(status, (int)MOBA_ERR_TIMEOUT);
 }
 
@@ -522,8 +580,20 @@ __global__ void __launch_bounds__(kQThreads, 1) bwd_q_tc_kernel(
       h = h_cur;
       r = valid ? (b * dm.N + t) * dm.hq + h : 0;
     }
-    load_half_row(base + kQOffQ, rho, hf, q + (size_t)r * kD, valid);
-    load_half_row(base + kQOffDO, rho, hf, dout + (size_t)r * kD, valid);
+    {
+      // this warp's 32 rows, half hf of each: four rows per copy instruction
+      // (eight lanes take a row's eight chunks of the half)
+      const int c8 = lane & 7;
+#pragma unroll
+      for (int k4 = 0; k4 < 8; ++k4) {
+        const int rl = 4 * k4 + (lane >> 3);
+        const int rs = __shfl_sync(0xffffffffu, r, rl);
+        const bool vs = __shfl_sync(0xffffffffu, valid, rl);
+        const uint32_t off = hf * kHalf + sw128_off(qd * 32 + rl, c8);
+        cp_async16(base + kQOffQ + off, q + (size_t)rs * kD + hf * 64 + c8 * 8, vs);
+        cp_async16(base + kQOffDO + off, dout + (size_t)rs * kD + hf * 64 + c8 * 8, vs);
+      }
+    }
     const float L2 = valid ? lse[((size_t)b * dm.hq + h) * dm.N + t] * kLog2e : INFINITY;
     const float Dr = valid ? delta[r] : 0.f;
     cp_async_commit();

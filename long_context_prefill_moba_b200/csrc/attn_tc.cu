@@ -221,11 +221,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         h = wk.h0 + w;
         r = valid ? (b * dm.N + t) * dm.hq + h : 0;
       }
+      // the warp copies its 32 rows two at a time: lanes 0-15 take the 16
+      // chunks of one row, lanes 16-31 those of the next, so each copy
+      // instruction reads two whole 256-byte rows instead of 16 bytes of 32
       const uint32_t qs = base + kOffQ + w * kTile;
-      const __nv_bfloat16* src = q + (size_t)r * kD;
+      {
+        const int wrow0 = (warp & 3) * 32, cc = lane & 15;
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        cp_async16(qs + (c >> 3) * kHalf + sw128_off(rho, c & 7), src + c * 8, valid);
+        for (int k2 = 0; k2 < 16; ++k2) {
+          const int rl = 2 * k2 + (lane >> 4);
+          const int rs = __shfl_sync(0xffffffffu, r, rl);
+          const bool vs = __shfl_sync(0xffffffffu, valid, rl);
+          cp_async16(qs + (cc >> 3) * kHalf + sw128_off(wrow0 + rl, cc & 7), q + (size_t)rs * kD + cc * 8, vs);
+        }
+      }
       cp_async_commit();
       cp_async_wait<0>();
       fence_proxy_async_smem();
