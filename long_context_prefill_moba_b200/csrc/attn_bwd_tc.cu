@@ -63,9 +63,10 @@ MOBA_DEV void red_add_v4(float* dst, float a, float b, float c, float d) {
 //   SMEM   the K and V tiles and four stages of q | dout row tiles (16 KB each).
 // The MMA issuer runs S^T, dP^T of row tile i and then dV, dK of tile i - 1,
 // so the elementwise warps work on one tile while the tensor core computes
-// the next; a gather warpgroup copies the rows of the tiles ahead (cp.async,
-// 16 bytes per request, three tiles in flight) with their lse, D and causal
-// limit.
+// the next.  Four gather warps copy the row tiles (cp.async) with their lse,
+// D and causal limit: warp w owns shared-memory stage w and the tiles
+// i = w mod 4, and publishes each tile as soon as its own copies have landed,
+// so four tiles are in flight.
 constexpr int kR = 64;                          // query rows per row tile
 constexpr int kStages = 4;                      // q | dout row-tile stages
 constexpr uint32_t kRHalf = kR * 128;           // 8 KB: one 64-column half of a row tile
@@ -76,8 +77,7 @@ constexpr int kKvWarps = kSoftmaxWarps + kGatherWarps + 1;   // elementwise, gat
 constexpr int kKvThreads = kKvWarps * 32;
 constexpr int kGatherWarp = kSoftmaxWarps;                    // first gather warp
 constexpr int kMmaWarp = kSoftmaxWarps + kGatherWarps;
-constexpr int kGatherLag = 2;          // row tiles in flight beyond the one published
-static_assert(kGatherLag <= kStages - 2, "the MMA must always find a published tile to proceed");
+static_assert(kGatherWarps == kStages, "each gather warp owns one row-tile stage");
 constexpr uint32_t kKvOffK = 0, kKvOffV = kTile, kKvOffQ = 2 * kTile;   // stage x at kKvOffQ + x kRStage
 constexpr uint32_t kKvSmem = 2 * kTile + kStages * kRStage + 1024;
 
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
   if (tid == 0) {
     mbar_init(bar(&ctl.kv_full), kGatherWarps);
     for (int x = 0; x < kStages; ++x) {
-      mbar_init(bar(&ctl.q_full[x]), kGatherWarps);
+      mbar_init(bar(&ctl.q_full[x]), 1);
       mbar_init(bar(&ctl.q_free[x]), 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -321,21 +321,17 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(&ctl.kv_full));
     }
-    // the warp's 16 rows of a row tile: lane l (and l + 16) holds row
-    // 16 gw + (l & 15) with its id, lse, D and causal limit.  The dependent
-    // loads are pipelined over the tiles: the row id of tile i + 2 (a read of
-    // `rows`), then lse and D of tile i + 1 (reads at that id), so that tile
-    // i's copies start without waiting on either.  Each copy instruction reads
-    // two whole 256-byte rows (lanes 0-15 one row's 16 chunks, 16-31 the next).
-    const int rr = 16 * gw + (lane & 15), cc = lane & 15;
+    // Row tiles i = gw, gw + 4, ... into stage gw.  Lane l holds rows l and
+    // l + 32 of the tile: id, lse, D and causal limit.  The row ids of the
+    // warp's next tile (a read of `rows`) load while this tile is copied; each
+    // copy instruction reads two whole 256-byte rows (lanes 0-15 one row's 16
+    // chunks, lanes 16-31 the next row's).
+    const int cc = lane & 15;
     struct RowOf {
       int r, t, h, tmax;
       bool valid;
     };
-    struct Scal {
-      float lse2, dlt;
-    };
-    auto row_of = [&](int i) -> RowOf {
+    auto row_of = [&](int i, int rr) -> RowOf {
       RowOf m{0, 0, 0, 0x7fffffff, false};
       if (i >= ntiles) return m;
       const RowTile rt = kv_row_tile(i, hist_tiles, offsets, dm, b, g, j, key0, pt, pr, pe);
@@ -352,64 +348,56 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
       }
       return m;
     };
-    auto scal_of = [&](RowOf& m) -> Scal {
-      Scal c{INFINITY, 0.f};
-      if (!m.valid) return c;
+    // lse (log2 units) and D of a row; +inf / 0 for no row
+    auto scal_of = [&](RowOf& m, float& lse2, float& dl) {
+      lse2 = INFINITY;
+      dl = 0.f;
+      if (!m.valid) return;
       if (m.t < 0) {
         m.h = m.r % dm.hq;
         m.t = (m.r / dm.hq) % dm.N;
       }
-      c.lse2 = lse[((size_t)b * dm.hq + m.h) * dm.N + m.t] * kLog2e;
-      c.dlt = delta[m.r];
-      return c;
+      lse2 = lse[((size_t)b * dm.hq + m.h) * dm.N + m.t] * kLog2e;
+      dl = delta[m.r];
     };
-    RowOf r0 = row_of(0), r1 = row_of(1);
-    Scal c0 = scal_of(r0);
+    const uint32_t sq = base + kKvOffQ + (uint32_t)gw * kRStage, sdo = sq + kRTile;
+    RowOf ra = row_of(gw, lane), rb = row_of(gw, lane + 32);
     bool ok = true;
-    int published = 0;
-    for (int i = 0; i < ntiles && ok; ++i) {
-      const int st = i % kStages;
-      // stage st held row tile i - kStages: free once its dV, dK MMAs completed
-      if (i >= kStages) ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.q_free[st]), ((i / kStages) - 1) & 1,
-                                                                abort_flag));
+    for (int i = gw, use = 0; i < ntiles && ok; i += kStages, ++use) {
+      // the stage held this warp's previous tile: free once its dV, dK MMAs completed
+      if (use >= 1) ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.q_free[gw]), (use - 1) & 1, abort_flag));
       if (!ok) break;
-      const RowOf r2 = row_of(i + 2);
-      const Scal c1 = scal_of(r1);
-      const uint32_t sq = base + kKvOffQ + (uint32_t)st * kRStage, sdo = sq + kRTile;
+      float la, da, lb, db;
+      scal_of(ra, la, da);
+      scal_of(rb, lb, db);
+      const RowOf na = row_of(i + kStages, lane), nb = row_of(i + kStages, lane + 32);
 #pragma unroll
-      for (int k2 = 0; k2 < 8; ++k2) {
-        const int rl = 2 * k2 + (lane >> 4);
-        const int rs = __shfl_sync(0xffffffffu, r0.r, rl);
-        const bool vs = __shfl_sync(0xffffffffu, r0.valid, rl);
-        const uint32_t off = (cc >> 3) * kRHalf + sw128_off(16 * gw + rl, cc & 7);
+      for (int k2 = 0; k2 < 32; ++k2) {
+        const int rl = 2 * k2 + (lane >> 4);     // row of the tile; its data sit in lane rl & 31
+        const int rsa = __shfl_sync(0xffffffffu, ra.r, rl & 31), rsb = __shfl_sync(0xffffffffu, rb.r, rl & 31);
+        const bool vsa = __shfl_sync(0xffffffffu, ra.valid, rl & 31),
+                   vsb = __shfl_sync(0xffffffffu, rb.valid, rl & 31);
+        const int rs = rl < 32 ? rsa : rsb;
+        const bool vs = rl < 32 ? vsa : vsb;
+        const uint32_t off = (cc >> 3) * kRHalf + sw128_off(rl, cc & 7);
         cp_async16(sq + off, q + (size_t)rs * kD + cc * 8, vs);
         cp_async16(sdo + off, dout + (size_t)rs * kD + cc * 8, vs);
       }
-      if (lane < 16) {
-        ctl.lse2[st][rr] = c0.lse2;
-        ctl.dlt[st][rr] = c0.dlt;
-        ctl.tmax[st][rr] = r0.tmax;
-      }
+      ctl.lse2[gw][lane] = la;
+      ctl.dlt[gw][lane] = da;
+      ctl.tmax[gw][lane] = ra.tmax;
+      ctl.lse2[gw][lane + 32] = lb;
+      ctl.dlt[gw][lane + 32] = db;
+      ctl.tmax[gw][lane + 32] = rb.tmax;
       cp_async_commit();
-      // row tile i - kGatherLag has landed once at most kGatherLag groups are pending
-      if (i >= kGatherLag) {
-        cp_async_wait<kGatherLag>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(&ctl.q_full[(i - kGatherLag) % kStages]));
-        published = i - kGatherLag + 1;
-      }
-      r0 = r1;
-      c0 = c1;
-      r1 = r2;
-    }
-    cp_async_wait<0>();
-    if (ok) {
+      cp_async_wait<0>();
       fence_proxy_async_smem();
       __syncwarp();
-      for (int i = published; i < ntiles; ++i)
-        if (lane == 0) mbar_arrive(bar(&ctl.q_full[i % kStages]));
+      if (lane == 0) mbar_arrive(bar(&ctl.q_full[gw]));
+      ra = na;
+      rb = nb;
     }
+    cp_async_wait<0>();
   } else if (lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idS = idesc_bf16(128, kR, false);     // A (K, V tile), B (q, dout rows) K-major
