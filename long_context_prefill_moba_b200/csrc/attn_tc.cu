@@ -110,6 +110,30 @@ struct Tile {
   int h0, t_first, t_last;   // kCur
 };
 
+// 32 rows of 256 bytes staged in shared memory: 16-byte chunk c of row rr at
+// rr * 256 + ((c ^ (rr & 15)) << 4), so that a warp writing one row per lane
+// and reading two rows per instruction both spread over the banks
+MOBA_DEV uint32_t stage_off(int rr, int c) { return (uint32_t)(rr * 256 + ((c ^ (rr & 15)) << 4)); }
+MOBA_DEV void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+// rows staged by the warp (lane i staged row i, destination row index `row`
+// of `dst`, 128 bf16 per row) written two whole rows per instruction
+MOBA_DEV void store_rows_from_stage(uint32_t stg, __nv_bfloat16* dst, int64_t row, bool valid, int lane) {
+  const int cc = lane & 15;
+#pragma unroll
+  for (int k2 = 0; k2 < 16; ++k2) {
+    const int rl = 2 * k2 + (lane >> 4);
+    const int64_t rd = __shfl_sync(0xffffffffu, (long long)row, rl);
+    const bool vd = __shfl_sync(0xffffffffu, valid, rl);
+    uint32_t x, y, z, w;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
+                 : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
+                 : "r"(stg + stage_off(rl, cc)));
+    if (vd) *reinterpret_cast<uint4*>(dst + rd * kD + cc * 8) = make_uint4(x, y, z, w);
+  }
+}
+
 template <int MODE>
 MOBA_DEV bool decode_tile(Tile& w, const int32_t* tile_start, const int32_t* offsets, const Dims& dm,
                           int ch) {
@@ -365,24 +389,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           const float inv = 1.f / l;
           // partials are kept in bf16 (the merge is done in fp32; the
           // rounding, 2^-9 relative of a normalised output, stays far below
-          // the output tolerance) to halve their HBM traffic
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(part_o) + pidx * kD;
+          // the output tolerance) to halve their HBM traffic.  Every MMA has
+          // completed, so each warp stages its 32 rows in its 8 KB of the Q
+          // buffers and stores two whole rows per instruction.
+          const uint32_t stg = base + kOffQ + (uint32_t)warp * 8192u;
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             uint32_t o[32];
             tmem_ld32(tO + cc * 32, o);
             tmem_wait_ld();
-            if (valid) {
-              uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
-              for (int e8 = 0; e8 < 4; ++e8)
-                d4[e8] = make_uint4(
-                    pack_bf16x2(__uint_as_float(o[8 * e8 + 0]) * inv, __uint_as_float(o[8 * e8 + 1]) * inv),
-                    pack_bf16x2(__uint_as_float(o[8 * e8 + 2]) * inv, __uint_as_float(o[8 * e8 + 3]) * inv),
-                    pack_bf16x2(__uint_as_float(o[8 * e8 + 4]) * inv, __uint_as_float(o[8 * e8 + 5]) * inv),
-                    pack_bf16x2(__uint_as_float(o[8 * e8 + 6]) * inv, __uint_as_float(o[8 * e8 + 7]) * inv));
-            }
+            for (int e8 = 0; e8 < 4; ++e8)
+              st_shared_v4(stg + stage_off(lane, cc * 4 + e8),
+                           pack_bf16x2(__uint_as_float(o[8 * e8 + 0]) * inv, __uint_as_float(o[8 * e8 + 1]) * inv),
+                           pack_bf16x2(__uint_as_float(o[8 * e8 + 2]) * inv, __uint_as_float(o[8 * e8 + 3]) * inv),
+                           pack_bf16x2(__uint_as_float(o[8 * e8 + 4]) * inv, __uint_as_float(o[8 * e8 + 5]) * inv),
+                           pack_bf16x2(__uint_as_float(o[8 * e8 + 6]) * inv, __uint_as_float(o[8 * e8 + 7]) * inv));
           }
+          __syncwarp();
+          store_rows_from_stage(stg, reinterpret_cast<__nv_bfloat16*>(part_o), (int64_t)pidx, valid, lane);
           if (valid) part_lse[pidx] = lse2;
         } else {
           // merge with the historical partials of the row (Algorithm 1 Step 4).
@@ -459,15 +484,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
             }
             __syncwarp();
           }
-          if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(out + (size_t)r * kD);
+          // out rows through the warp's (now idle) staging slot 0: two whole
+          // rows per store instruction
 #pragma unroll
-            for (int e8 = 0; e8 < 16; ++e8)
-              d4[e8] = make_uint4(pack_bf16x2(acc[8 * e8 + 0], acc[8 * e8 + 1]),
-                                  pack_bf16x2(acc[8 * e8 + 2], acc[8 * e8 + 3]),
-                                  pack_bf16x2(acc[8 * e8 + 4], acc[8 * e8 + 5]),
-                                  pack_bf16x2(acc[8 * e8 + 6], acc[8 * e8 + 7]));
-          }
+          for (int e8 = 0; e8 < 16; ++e8)
+            st_shared_v4(stage + stage_off(lane, e8), pack_bf16x2(acc[8 * e8 + 0], acc[8 * e8 + 1]),
+                         pack_bf16x2(acc[8 * e8 + 2], acc[8 * e8 + 3]), pack_bf16x2(acc[8 * e8 + 4], acc[8 * e8 + 5]),
+                         pack_bf16x2(acc[8 * e8 + 6], acc[8 * e8 + 7]));
+          __syncwarp();
+          store_rows_from_stage(stage, out, (int64_t)r, valid, lane);
           if (valid && lse != nullptr)
             lse[((size_t)b * dm.hq + h) * dm.N + t] = (M + log2f(W)) * kLn2;
         }
