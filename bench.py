@@ -59,21 +59,31 @@ def routed_flops(cfg, routed_pairs: int) -> float:
     return 4.0 * cfg.head_dim * (routed_pairs * cfg.block + cur * cfg.batch * cfg.hq)
 
 
+ATTN_SOURCES = ("attn_tc.cu", "attn_pair_tc.cu")
+
+
+def attention_source_sha() -> str:
+    """sha256 of the attention kernels' sources (csrc/attn_tc.cu, then
+    csrc/attn_pair_tc.cu), which the traffic record is tied to."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "long_context_prefill_moba_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def recorded_traffic(rows_per_layer: int):
     """DRAM bytes of one attention step (moba_attn_fwd) from the committed ncu
     capture (profiles/attn_traffic.json), scaled by the rows the gate routes
     (the partial results and the gathered q rows dominate and grow with them).
     None when the attention kernels changed since the capture."""
-    import hashlib
     p = os.path.join(ROOT, "profiles", "attn_traffic.json")
     if not os.path.exists(p):
         return None, "no capture"
     with open(p) as f:
         d = json.load(f)
-    src = os.path.join(ROOT, "long_context_prefill_moba_b200", "csrc", "attn_tc.cu")
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    if sha != d.get("kernel_source_sha256"):
+    if attention_source_sha() != d.get("kernel_source_sha256"):
         return None, "kernel changed since the capture"
     return d["dram_bytes_per_row"] * rows_per_layer, (
         f"ncu capture of the {d['config']} layer ({d['dram_bytes_per_layer'] / 1e9:.2f} GB), "

@@ -570,14 +570,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       for (int i = 0; i < nkt && ok; ++i) {
         const int s = i & 1, s1 = (i + 1) & 1;
         const bool more = i + 1 < nkt;
+        // the K/V tiles are normally resident long before P0: their barriers
+        // are waited for first, so that PV0 and S0 go out back to back
         ok = mbar_wait(bar(&ctl.v_full[s]), (i >> 1) & 1, abort_flag) &&
+             (!more || mbar_wait(bar(&ctl.k_full[s1]), ((i + 1) >> 1) & 1, abort_flag)) &&
              mbar_wait(bar(&ctl.p_full[0]), i & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         issue_pv(0, s, i > 0);
         if (more) {
-          if (!(ok = mbar_wait(bar(&ctl.k_full[s1]), ((i + 1) >> 1) & 1, abort_flag))) break;
-          tc_fence_after();
           issue_s(0, s1);
           mma_commit(bar(&ctl.s_full[0]));
         }
@@ -677,9 +678,17 @@ cudaError_t launch_tc(const Dims& dm, const void* q, const void* k, const void* 
 
 int attn_tc_rows_per_tile() { return kRowsPerCta; }
 
+// the CTA-pair historical kernel (csrc/attn_pair_tc.cu) takes the same 256-row tiles
+bool attn_hist_pair_enabled();
+cudaError_t launch_attn_pair_hist(const Dims& dm, const void* q, const void* k, const void* v,
+                                  const int32_t* sel, const int32_t* offsets, const int32_t* rows,
+                                  const AttnWs& ws, int ch, int64_t grid, cudaStream_t stream);
+
 cudaError_t launch_attn_tc_hist(const Dims& dm, const void* q, const void* k, const void* v,
                                 const int32_t* sel, const int32_t* offsets, const int32_t* rows,
                                 const AttnWs& ws, int ch, int64_t grid, cudaStream_t stream) {
+  if (attn_hist_pair_enabled())
+    return launch_attn_pair_hist(dm, q, k, v, sel, offsets, rows, ws, ch, grid, stream);
   return launch_tc<kHist>(dm, q, k, v, sel, offsets, rows, ws, nullptr, nullptr, ch, grid, stream);
 }
 

@@ -117,6 +117,70 @@ MOBA_DEV void mma_commit(uint32_t bar) {
                : "memory");
 }
 
+// ---- CTA pairs: a cluster of two CTAs issuing one tcgen05 MMA together ------
+// (.cta_group::2: M = 256 rows, 128 in each CTA's TMEM lanes; each CTA's
+// shared memory holds its own 128 rows of A and half of B's N columns at the
+// same offset; every tcgen05 alloc / MMA / commit of such a kernel is
+// .cta_group::2, issued by the even CTA of the pair)
+MOBA_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+// address of the same shared variable in CTA `rank` of the cluster
+MOBA_DEV uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(d) : "r"(addr), "r"(rank));
+  return d;
+}
+// arrive on an mbarrier given by its cluster address (own CTA or the peer);
+// default semantics, as in CUTLASS's cluster pipelines: the TMEM and shared
+// memory handed over are ordered by tcgen05 / proxy fences before the arrive
+MOBA_DEV void mbar_arrive_cluster(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];\n" ::"r"(cl_addr) : "memory");
+}
+// every thread of both CTAs
+MOBA_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+MOBA_DEV void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {   // one warp of each CTA
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst_smem),
+               "r"(ncols));
+}
+MOBA_DEV void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::);
+}
+MOBA_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols));
+}
+MOBA_DEV void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+MOBA_DEV void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// arrive on the barrier at this shared offset in the issuing CTA only
+MOBA_DEV void mma_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+               : "memory");
+}
+// arrive on the barrier at this shared offset in both CTAs of the pair
+MOBA_DEV void mma_commit_pair_both(uint32_t bar) {
+  const uint16_t mask = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator.
 // bits [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
 // 15 A major (0 = K), 16 B major (1 = MN), [17,23) N >> 3, [24,29) M >> 4.

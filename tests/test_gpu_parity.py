@@ -218,3 +218,34 @@ def test_convenience_forward_matches_layer(cuda_device):
     torch.cuda.synchronize()
     assert torch.equal(out, res["out"])
     assert torch.equal(lse, res["lse"])
+
+
+# The historical-block kernel on CTA pairs (tcgen05 .cta_group::2, M = 256 over
+# two SMs, selectable with MOBA_HIST_KERNEL=pair) against the oracle: several
+# passes, blocks that are not a multiple of the key tile, GQA 8, and a sampled
+# 131072-token layer with gate scores in the hundreds.
+PAIR = {
+    "mqar": (S.get_config("mqar"), 0, 0.0),
+    "ragged_multipass": (EDGE["ragged_multipass"], CHUNK["ragged_multipass"], 0.0),
+    "gqa8_bf16": (EDGE["gqa8_bf16"], CHUNK["gqa8_bf16"], 0.0),
+    "odd_block_multipass": (S.get_config("mqar").replace(batch=2, seqlen=5000, hq=4, hkv=2, block=320,
+                                                         topk=4), 2048, 0.0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PAIR))
+def test_pair_kernel_full(cuda_device, monkeypatch, name):
+    monkeypatch.setenv("MOBA_HIST_KERNEL", "pair")
+    cfg, chunk, rel = PAIR[name]
+    res = run_gpu(cfg, query_chunk=chunk)
+    info = full_parity(cfg, res, rel=rel)
+    print("pair", name, info)
+
+
+def test_pair_kernel_128k_large_scores_sampled(cuda_device, monkeypatch):
+    monkeypatch.setenv("MOBA_HIST_KERNEL", "pair")
+    cfg = S.get_config("llama8b_128k").replace(**LARGE)
+    res = run_gpu(cfg)
+    worst = sampled_parity(cfg, res, sampled_rows(cfg, 128, seed=11, chunk=_chunk(res)), rel=LARGE_REL)
+    assert res["layer"].device_status() == (0, 0)
+    print("pair llama8b_128k large scores worst", worst)

@@ -50,13 +50,13 @@ def test_single_rank_is_identity():
 
 
 def test_traffic_record_matches_the_attention_source():
-    # bench.py reports the ncu-measured DRAM traffic only while csrc/attn_tc.cu is
-    # the source it was captured from; a kernel edit must come with a new capture
-    import hashlib
+    # bench.py reports the ncu-measured DRAM traffic only while the attention
+    # kernels' sources are the ones it was captured from; a kernel edit must
+    # come with a new capture
     import json
     import os
+    import bench
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     rec = json.load(open(os.path.join(root, "profiles", "attn_traffic.json")))
-    src = open(os.path.join(root, "long_context_prefill_moba_b200", "csrc", "attn_tc.cu"), "rb").read()
-    assert hashlib.sha256(src).hexdigest() == rec["kernel_source_sha256"]
+    assert bench.attention_source_sha() == rec["kernel_source_sha256"]
     assert 0 < rec["dram_bytes_per_row"] < 4096
