@@ -471,11 +471,15 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_kv_tc_kernel(
 // ============================================================================ dQ
 constexpr int kHist = 0, kCur = 1;
 constexpr int kQThreads = (kSoftmaxWarps + 2) * 32;   // softmax, TMA producer, MMA issuer
-constexpr uint32_t kQOffQ = 0, kQOffDO = kTile, kQOffK = 2 * kTile, kQOffV = 4 * kTile;
-constexpr uint32_t kQSmem = 6 * kTile + 1024;
+// K tiles in three stages: K(i) is read by dQ(i), the last MMA of tile i, and
+// K(i + 3) must already be arriving when S(i + 3) is issued during tile i + 2
+constexpr int kQKStages = 3;
+constexpr uint32_t kQOffQ = 0, kQOffDO = kTile, kQOffK = 2 * kTile, kQOffV = (2 + kQKStages) * kTile;
+constexpr uint32_t kQSmem = (4 + kQKStages) * kTile + 1024;
 
 struct QCtl {
-  uint64_t q_full, k_full[2], v_full[2], k_free[2], v_free[2], s_full, p_full, o_full, drain;
+  uint64_t q_full, k_full[kQKStages], v_full[2], k_free[kQKStages], v_free[2], s_full, s_read, p_full[2], o_full,
+      drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -527,14 +531,18 @@ __global__ void __launch_bounds__(kQThreads, 1) bwd_q_tc_kernel(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     mbar_init(bar(&ctl.q_full), kSoftmaxWarps);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kQKStages; ++s) {
       mbar_init(bar(&ctl.k_full[s]), 1);
-      mbar_init(bar(&ctl.v_full[s]), 1);
       mbar_init(bar(&ctl.k_free[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(&ctl.v_full[s]), 1);
       mbar_init(bar(&ctl.v_free[s]), 1);
     }
     mbar_init(bar(&ctl.s_full), 1);
-    mbar_init(bar(&ctl.p_full), kSoftmaxWarps);
+    mbar_init(bar(&ctl.s_read), kSoftmaxWarps);
+    mbar_init(bar(&ctl.p_full[0]), kSoftmaxWarps);
+    mbar_init(bar(&ctl.p_full[1]), kSoftmaxWarps);
     mbar_init(bar(&ctl.o_full), 1);
     mbar_init(bar(&ctl.drain), 1);
     ctl.abort = 0;
@@ -597,12 +605,18 @@ __global__ void __launch_bounds__(kQThreads, 1) bwd_q_tc_kernel(
       ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.s_full), i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
+      // dP(i), then dS(i), in columns [128, 256) for even i, [384, 512) for odd i
+      const uint32_t tD = tb + ((i & 1) ? 384u : 128u) + 64u * hf + lane_off;
       uint32_t sr[64], dr[64];
       tmem_ld32(tb + 64u * hf + lane_off, sr);
       tmem_ld32(tb + 64u * hf + 32 + lane_off, sr + 32);
-      tmem_ld32(tb + 128u + 64u * hf + lane_off, dr);
-      tmem_ld32(tb + 128u + 64u * hf + 32 + lane_off, dr + 32);
+      tmem_ld32(tD, dr);
+      tmem_ld32(tD + 32, dr + 32);
       tmem_wait_ld();
+      // S(i) is in registers: the MMA issuer may compute S(i+1) over it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(&ctl.s_read));
       const int u0 = key0 + i * kT + 64 * hf;     // key of column 0 of this warp's half
       const int vlo = lo_u - u0, vhi = hi_u - u0;
       uint32_t ps[32];
@@ -615,11 +629,11 @@ __global__ void __launch_bounds__(kQThreads, 1) bwd_q_tc_kernel(
         ps[c] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * c]) - Dr), p1 * (__uint_as_float(dr[2 * c + 1]) - Dr));
       }
       // dS over this warp's own dP columns [64 hf, 64 hf + 32): already read
-      tmem_st32(tb + 128u + 64u * hf + lane_off, ps);
+      tmem_st32(tD, ps);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(&ctl.p_full));
+      if (lane == 0) mbar_arrive(bar(&ctl.p_full[i & 1]));
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(&ctl.o_full), 0, abort_flag));
     if (ok) {
@@ -649,12 +663,12 @@ __global__ void __launch_bounds__(kQThreads, 1) bwd_q_tc_kernel(
       const int x0 = g * kD;
       int issued_k = 0, issued_v = 0;
       for (int i = 0; i < nkt; ++i) {
-        const int s = i & 1;
-        const uint32_t ks = base + kQOffK + s * kTile, vs = base + kQOffV + s * kTile;
-        if (i >= 2 && !mbar_wait(bar(&ctl.k_free[s]), ((i >> 1) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(&ctl.k_full[s]), kTile);
-        tma_load_2d(ks, &tmK, x0, y0 + i * kT, bar(&ctl.k_full[s]));
-        tma_load_2d(ks + kHalf, &tmK, x0 + 64, y0 + i * kT, bar(&ctl.k_full[s]));
+        const int sk = i % kQKStages, uk = i / kQKStages, s = i & 1;
+        const uint32_t ks = base + kQOffK + sk * kTile, vs = base + kQOffV + s * kTile;
+        if (i >= kQKStages && !mbar_wait(bar(&ctl.k_free[sk]), (uk - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(&ctl.k_full[sk]), kTile);
+        tma_load_2d(ks, &tmK, x0, y0 + i * kT, bar(&ctl.k_full[sk]));
+        tma_load_2d(ks + kHalf, &tmK, x0 + 64, y0 + i * kT, bar(&ctl.k_full[sk]));
         issued_k = i + 1;
         if (i >= 2 && !mbar_wait(bar(&ctl.v_free[s]), ((i >> 1) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(&ctl.v_full[s]), kTile);
@@ -664,8 +678,8 @@ __global__ void __launch_bounds__(kQThreads, 1) bwd_q_tc_kernel(
       }
       if (*abort_flag) {
         int never = 0;
-        for (int i = (issued_k > 2 ? issued_k - 2 : 0); i < issued_k; ++i)
-          mbar_wait(bar(&ctl.k_full[i & 1]), (i >> 1) & 1, &never);
+        for (int i = (issued_k > kQKStages ? issued_k - kQKStages : 0); i < issued_k; ++i)
+          mbar_wait(bar(&ctl.k_full[i % kQKStages]), (i / kQKStages) & 1, &never);
         for (int i = (issued_v > 2 ? issued_v - 2 : 0); i < issued_v; ++i)
           mbar_wait(bar(&ctl.v_full[i & 1]), (i >> 1) & 1, &never);
       }
@@ -678,14 +692,11 @@ __global__ void __launch_bounds__(kQThreads, 1) bwd_q_tc_kernel(
     const uint32_t loQ = sdesc_lo(base + kQOffQ, 16), loDO = sdesc_lo(base + kQOffDO, 16),
                    loK = sdesc_lo(base + kQOffK, 16), loV = sdesc_lo(base + kQOffV, 16),
                    mnK = sdesc_lo(base + kQOffK, kHalf);
-    bool ok = mbar_wait(bar(&ctl.q_full), 0, abort_flag);
-    for (int i = 0; i < nkt && ok; ++i) {
-      const int s = i & 1;
-      ok = mbar_wait(bar(&ctl.k_full[s]), (i >> 1) & 1, abort_flag) &&
-           mbar_wait(bar(&ctl.v_full[s]), (i >> 1) & 1, abort_flag);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t ko = s ? (kTile >> 4) : 0u;
+    // S(n) into columns [0, 128) and dP(n) into its buffer, [128, 256) for even
+    // n and [384, 512) for odd n (dQ accumulates in [256, 384))
+    auto issue_sdp = [&](int n) {
+      const uint32_t ko = (uint32_t)(n % kQKStages) * (kTile >> 4), vo = (n & 1) ? (kTile >> 4) : 0u;
+      const uint32_t tdp = tb + ((n & 1) ? 384u : 128u);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
@@ -694,19 +705,44 @@ __global__ void __launch_bounds__(kQThreads, 1) bwd_q_tc_kernel(
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-        mma_ss(tb + 128u, sdesc_join(loDO + off, hi), sdesc_join(loV + ko + off, hi), idS, kk > 0);
+        mma_ss(tdp, sdesc_join(loDO + off, hi), sdesc_join(loV + vo + off, hi), idS, kk > 0);
       }
-      mma_commit(bar(&ctl.s_full));
-      mma_commit(bar(&ctl.v_free[s]));
-      if (!(ok = mbar_wait(bar(&ctl.p_full), i & 1, abort_flag))) break;
+    };
+    auto kv_ready = [&](int n) -> bool {
+      return mbar_wait(bar(&ctl.k_full[n % kQKStages]), (n / kQKStages) & 1, abort_flag) &&
+             mbar_wait(bar(&ctl.v_full[n & 1]), (n >> 1) & 1, abort_flag);
+    };
+    bool ok = mbar_wait(bar(&ctl.q_full), 0, abort_flag) && kv_ready(0);
+    if (ok) {
       tc_fence_after();
-      // dQ += dS K: dS of keys 0-63 in columns 128-159, keys 64-127 in 192-223
+      issue_sdp(0);
+      mma_commit(bar(&ctl.s_full));
+      mma_commit(bar(&ctl.v_free[0]));
+    }
+    for (int i = 0; i < nkt && ok; ++i) {
+      // S(i+1), dP(i+1) as soon as the softmax warps hold S(i) in registers: they
+      // run on the tensor cores while dS(i) is computed (dP(i+1) goes to the
+      // other buffer; the one it overwrites was last read by dQ(i-1), issued
+      // before it)
+      if (i + 1 < nkt) {
+        if (!(ok = kv_ready(i + 1) && mbar_wait(bar(&ctl.s_read), i & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_sdp(i + 1);
+        mma_commit(bar(&ctl.s_full));
+        mma_commit(bar(&ctl.v_free[(i + 1) & 1]));
+      }
+      if (!(ok = mbar_wait(bar(&ctl.p_full[i & 1]), (i >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      // dQ += dS K: dS of keys 0-63 in the first 32 columns of its buffer, keys
+      // 64-127 in columns 64-95
+      const uint32_t ko = (uint32_t)(i % kQKStages) * (kTile >> 4);
+      const uint32_t tds = tb + ((i & 1) ? 384u : 128u);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t a = tb + 128u + (kk < 4 ? kk * 8u : 64u + (kk - 4) * 8u);
+        const uint32_t a = tds + (kk < 4 ? kk * 8u : 64u + (kk - 4) * 8u);
         mma_ts(tb + 256u, a, sdesc_join(mnK + ko + ((kk * 2048) >> 4), hi), idQ, (i > 0 || kk > 0) ? 1u : 0u);
       }
-      mma_commit(bar(&ctl.k_free[s]));
+      mma_commit(bar(&ctl.k_free[i % kQKStages]));
     }
     if (ok) {
       mma_commit(bar(&ctl.o_full));
