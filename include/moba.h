@@ -105,8 +105,9 @@ MOBA_API int64_t moba_num_blocks(const moba_shape_t* shape);
  * results of one pass fit a bounded workspace.  query_chunk > 0 (a multiple
  * of 128) is used as given; 0 picks the largest power of two >= 128 whose
  * partials fit 8 GiB, capped at seqlen rounded up to 128 (a partial takes
- * 2 * head_dim + 4 bytes on the tensor-core path, bf16 with head_dim 128, and
- * 4 * (head_dim + 1) bytes otherwise; 65536 tokens at 1M, 524288 at 10M). */
+ * 2 * head_dim + 4 bytes on the tensor-core path, bf16 with head_dim 128 or
+ * 64, and 4 * (head_dim + 1) bytes for fp32; 65536 tokens at 1M, 524288 at
+ * 10M). */
 MOBA_API int64_t moba_query_chunk(const moba_shape_t* shape);
 
 /* Number of passes: ceil(seqlen / C). */

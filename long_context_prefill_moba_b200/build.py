@@ -11,7 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoba.so")
-SOURCES = ["moba_api.cu", "meanpool.cu", "gate.cu", "attn.cu", "attn_mma.cu", "attn_f32.cu", "attn_tc.cu", "attn_pair_tc.cu", "attn_bwd.cu", "attn_bwd_tc.cu", "gate_tc.cu", "gate_pooled.cu", "index_check.cu", "selftest.cu"]
+SOURCES = ["moba_api.cu", "meanpool.cu", "gate.cu", "attn.cu", "attn_f32.cu", "attn_tc.cu", "attn_pair_tc.cu", "attn_bwd.cu", "attn_bwd_tc.cu", "gate_tc.cu", "gate_pooled.cu", "index_check.cu", "selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
          "-Xcompiler", "-fvisibility=hidden", "-Xptxas", "-O3"]

@@ -1,5 +1,5 @@
 // K3 on 5th-generation tensor cores (tcgen05 + TMEM + TMA): the two attention
-// steps of MoBA for bf16, head_dim 128.
+// steps of MoBA for bf16, head_dim D = 128 or 64.
 //
 // "MoBA: Mixture of Block Attention for Long-Context LLMs", paper-graph summary
 // §3 "The Core MoBA Attention Equation" (Softmax(q K[I]^T) V[I]), "Causality
@@ -28,9 +28,10 @@
 // Per 128-key tile i: S_w = Q_w K_i^T (SS MMA, fp32 in TMEM), the softmax warps
 // read S_w, keep a lazily rescaled running max, write P_w = exp2(S - m) as bf16
 // back over S_w, and O_w += P_w V_i runs as a TS MMA (A operand from TMEM).
-// TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) columns.
-// SMEM: Q0 Q1 (32 KB each), K and V double buffered (32 KB per tile): 192 KB.
-// All tiles use the 128-byte swizzled K-major layout (V is read MN-major).
+// TMEM: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D) columns.
+// SMEM: Q0 Q1, K and V double buffered, each tile 128 rows x D (32 KB for
+// D = 128, 16 KB for D = 64): 192 or 96 KB.  All tiles use the 128-byte
+// swizzled K-major layout in 64-column halves (V is read MN-major).
 //
 // The MMA issue order per tile i is PV0_i, S0_{i+1}, PV1_i, S1_{i+1}; tcgen05
 // operations of one thread execute in order and a commit covers every earlier
@@ -52,7 +53,6 @@ using namespace sm100;
 
 constexpr int kHist = 0, kCur = 1;
 
-constexpr int kD = 128;
 constexpr int kQT = 128;                 // rows per Q tile
 constexpr int kBK = 128;                 // keys per K/V tile
 constexpr int kRowsPerCta = 2 * kQT;
@@ -62,12 +62,7 @@ constexpr int kSoftmaxRegs = 216;
 constexpr int kServiceRegs = 64;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kServiceRegs <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr uint32_t kTile = kBK * kD * 2; // 32 KB, two 16 KB column halves
-constexpr uint32_t kHalf = 16384;
-constexpr uint32_t kOffQ = 0;            // Q0 at 0, Q1 at kTile
-constexpr uint32_t kOffK = 2 * kTile;    // stages at +0, +kTile
-constexpr uint32_t kOffV = 4 * kTile;
-constexpr uint32_t kSmemBytes = 6 * kTile + 1024;
+constexpr uint32_t kHalf = 16384;       // a 64-column half of a 128-row tile (128-byte rows)
 constexpr float kRescaleThreshold = 8.f; // log2 units: rescale O only when the max grows by > 2^8
 // A tile whose probabilities, taken against the row's current base, sum to at
 // most 2^15 (so none exceeds 2^15) is accepted without computing its row max.
@@ -81,11 +76,26 @@ constexpr float kFastSumLimit = 32768.f;
 constexpr int kPolyOf8 = MOBA_POLY_OF8;
 static_assert(kPolyOf8 >= 0 && kPolyOf8 <= 8, "pairs per 8");
 // merge staging in the current-block epilogue: per softmax warp kMergeStages
-// slots of 32 rows x 256 bytes; the 8 warps' stages fill the Q/K/V buffers
+// slots of 32 rows; the 8 warps' stages fill the Q/K/V buffers
 constexpr int kMergeStages = 3;
-constexpr uint32_t kMergeSlotBytes = 32 * kD * 2;
-constexpr uint32_t kMergeWarpBytes = kMergeStages * kMergeSlotBytes;
-static_assert(8 * kMergeWarpBytes <= 6 * kTile, "merge staging exceeds the tile buffers");
+
+// Shared-memory geometry for head_dim D (64 or 128).  Q, K and V tiles are 128
+// rows of D bf16, stored as D / 64 column halves of 128-byte rows (16 KB
+// each), 128-byte swizzled; Q0 Q1 at 0, K stages at 2 tiles, V stages at 4.
+template <int D>
+struct Geo {
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static constexpr uint32_t kTile = kBK * D * 2;
+  static constexpr int kHalves = D / 64;
+  static constexpr uint32_t kOffQ = 0, kOffK = 2 * kTile, kOffV = 4 * kTile;
+  static constexpr uint32_t kSmem = 6 * kTile + 1024;
+  static constexpr int kRowBytes = 2 * D;           // one bf16 row
+  static constexpr int kChunks = D / 8;             // its 16-byte chunks
+  static constexpr int kRowsPerOp = 32 / kChunks;   // rows one warp instruction covers
+  static constexpr uint32_t kMergeSlot = 32 * kRowBytes;
+  static constexpr uint32_t kMergeWarp = kMergeStages * kMergeSlot;
+  static_assert(8 * kMergeWarp <= 6 * kTile, "merge staging exceeds the tile buffers");
+};
 // MUFU exponential: 1 = ex2.approx.ftz.f32 directly, 0 = exp2f
 #ifndef MOBA_EX2_DIRECT
 #define MOBA_EX2_DIRECT 1
@@ -110,27 +120,33 @@ struct Tile {
   int h0, t_first, t_last;   // kCur
 };
 
-// 32 rows of 256 bytes staged in shared memory: 16-byte chunk c of row rr at
-// rr * 256 + ((c ^ (rr & 15)) << 4), so that a warp writing one row per lane
-// and reading two rows per instruction both spread over the banks
-MOBA_DEV uint32_t stage_off(int rr, int c) { return (uint32_t)(rr * 256 + ((c ^ (rr & 15)) << 4)); }
+// 32 rows of D bf16 staged in shared memory: 16-byte chunk c of row rr at
+// rr * 2D + ((c ^ (rr mod D/8)) << 4), so that a warp writing one row per lane
+// and reading whole rows (two or four per instruction) both spread over the banks
+template <int D>
+MOBA_DEV uint32_t stage_off(int rr, int c) {
+  return (uint32_t)(rr * Geo<D>::kRowBytes + ((c ^ (rr & (Geo<D>::kChunks - 1))) << 4));
+}
 MOBA_DEV void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
 // rows staged by the warp (lane i staged row i, destination row index `row`
-// of `dst`, 128 bf16 per row) written two whole rows per instruction
+// of `dst`, D bf16 per row) written whole rows at a time (two per instruction
+// for D = 128, four for D = 64)
+template <int D>
 MOBA_DEV void store_rows_from_stage(uint32_t stg, __nv_bfloat16* dst, int64_t row, bool valid, int lane) {
-  const int cc = lane & 15;
+  using G = Geo<D>;
+  const int cc = lane % G::kChunks;
 #pragma unroll
-  for (int k2 = 0; k2 < 16; ++k2) {
-    const int rl = 2 * k2 + (lane >> 4);
+  for (int k2 = 0; k2 < 32 / G::kRowsPerOp; ++k2) {
+    const int rl = G::kRowsPerOp * k2 + lane / G::kChunks;
     const int64_t rd = __shfl_sync(0xffffffffu, (long long)row, rl);
     const bool vd = __shfl_sync(0xffffffffu, valid, rl);
     uint32_t x, y, z, w;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n"
                  : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
-                 : "r"(stg + stage_off(rl, cc)));
-    if (vd) *reinterpret_cast<uint4*>(dst + rd * kD + cc * 8) = make_uint4(x, y, z, w);
+                 : "r"(stg + stage_off<D>(rl, cc)));
+    if (vd) *reinterpret_cast<uint4*>(dst + rd * D + cc * 8) = make_uint4(x, y, z, w);
   }
 }
 
@@ -178,7 +194,7 @@ MOBA_DEV bool decode_tile(Tile& w, const int32_t* tile_start, const int32_t* off
   return true;
 }
 
-template <int MODE>
+template <int MODE, int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ sel,
@@ -186,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const int32_t* __restrict__ tile_start, float* __restrict__ part_o,
     float* __restrict__ part_lse, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
     int* __restrict__ status, Dims dm, int ch) {
+  using G = Geo<D>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ Ctl ctl;
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -245,18 +262,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         h = wk.h0 + w;
         r = valid ? (b * dm.N + t) * dm.hq + h : 0;
       }
-      // the warp copies its 32 rows two at a time: lanes 0-15 take the 16
-      // chunks of one row, lanes 16-31 those of the next, so each copy
-      // instruction reads two whole 256-byte rows instead of 16 bytes of 32
-      const uint32_t qs = base + kOffQ + w * kTile;
+      // the warp copies its 32 rows whole rows at a time: for D = 128 lanes
+      // 0-15 take the 16 chunks of one row and lanes 16-31 those of the next
+      // (four rows of 8 chunks for D = 64), so each copy instruction reads
+      // whole rows instead of 16 bytes of 32 rows
+      const uint32_t qs = base + G::kOffQ + w * G::kTile;
       {
-        const int wrow0 = (warp & 3) * 32, cc = lane & 15;
+        const int wrow0 = (warp & 3) * 32, cc = lane % G::kChunks;
 #pragma unroll
-        for (int k2 = 0; k2 < 16; ++k2) {
-          const int rl = 2 * k2 + (lane >> 4);
+        for (int k2 = 0; k2 < 32 / G::kRowsPerOp; ++k2) {
+          const int rl = G::kRowsPerOp * k2 + lane / G::kChunks;
           const int rs = __shfl_sync(0xffffffffu, r, rl);
           const bool vs = __shfl_sync(0xffffffffu, valid, rl);
-          cp_async16(qs + (cc >> 3) * kHalf + sw128_off(wrow0 + rl, cc & 7), q + (size_t)rs * kD + cc * 8, vs);
+          cp_async16(qs + (cc >> 3) * kHalf + sw128_off(wrow0 + rl, cc & 7), q + (size_t)rs * D + cc * 8, vs);
         }
       }
       cp_async_commit();
@@ -352,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
             // S_i complete implies PV_(i-1) complete (MMA issue order), so O is final here
             const float f = need ? exp2f(m_used - mxs) : 1.f;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < D / 32; ++cc) {
               uint32_t o[32];
               tmem_ld32(tO + cc * 32, o);
               tmem_wait_ld();
@@ -392,22 +410,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           // the output tolerance) to halve their HBM traffic.  Every MMA has
           // completed, so each warp stages its 32 rows in its 8 KB of the Q
           // buffers and stores two whole rows per instruction.
-          const uint32_t stg = base + kOffQ + (uint32_t)warp * 8192u;
+          const uint32_t stg = base + G::kOffQ + (uint32_t)warp * (32u * G::kRowBytes);
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
+          for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
             tmem_ld32(tO + cc * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e8 = 0; e8 < 4; ++e8)
-              st_shared_v4(stg + stage_off(lane, cc * 4 + e8),
+              st_shared_v4(stg + stage_off<D>(lane, cc * 4 + e8),
                            pack_bf16x2(__uint_as_float(o[8 * e8 + 0]) * inv, __uint_as_float(o[8 * e8 + 1]) * inv),
                            pack_bf16x2(__uint_as_float(o[8 * e8 + 2]) * inv, __uint_as_float(o[8 * e8 + 3]) * inv),
                            pack_bf16x2(__uint_as_float(o[8 * e8 + 4]) * inv, __uint_as_float(o[8 * e8 + 5]) * inv),
                            pack_bf16x2(__uint_as_float(o[8 * e8 + 6]) * inv, __uint_as_float(o[8 * e8 + 7]) * inv));
           }
           __syncwarp();
-          store_rows_from_stage(stg, reinterpret_cast<__nv_bfloat16*>(part_o), (int64_t)pidx, valid, lane);
+          store_rows_from_stage<D>(stg, reinterpret_cast<__nv_bfloat16*>(part_o), (int64_t)pidx, valid, lane);
           if (valid) part_lse[pidx] = lse2;
         } else {
           // merge with the historical partials of the row (Algorithm 1 Step 4).
@@ -430,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           for (int s = 0; s < MOBA_MAX_TOPK - 1; ++s) W += exp2f(pl[s] - M);
           const float iw = 1.f / W;
           const float fc = wc / l * iw;
-          float acc[kD];
+          float acc[D];
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
+          for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
             tmem_ld32(tO + cc * 32, o);
             tmem_wait_ld();
@@ -441,18 +459,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           }
           fence_proxy_async_smem();
           const int nhw = __reduce_max_sync(0xffffffffu, nh);
-          const uint32_t stage = base + (uint32_t)warp * kMergeWarpBytes;
+          const uint32_t stage = base + (uint32_t)warp * G::kMergeWarp;
           const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(part_o);
           // row rr of this warp is token t - lane + rr: its partials start rr * hq * KH slots later
           const size_t pbase0 = pbase - (size_t)lane * dm.hq * KH;
           auto issue = [&](int sl) {
-            const uint32_t buf = stage + (uint32_t)(sl % kMergeStages) * kMergeSlotBytes;
+            const uint32_t buf = stage + (uint32_t)(sl % kMergeStages) * G::kMergeSlot;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const int rr = 2 * k + (lane >> 4), c = lane & 15;
+            for (int k = 0; k < 32 / G::kRowsPerOp; ++k) {
+              const int rr = G::kRowsPerOp * k + lane / G::kChunks, c = lane % G::kChunks;
               const bool live = sl < __shfl_sync(0xffffffffu, nh, rr);
-              const __nv_bfloat16* src = live ? pb + (pbase0 + (size_t)rr * dm.hq * KH + sl) * kD + c * 8 : pb;
-              cp_async16(buf + rr * 256 + ((c ^ (rr & 15)) << 4), src, live);
+              const __nv_bfloat16* src = live ? pb + (pbase0 + (size_t)rr * dm.hq * KH + sl) * D + c * 8 : pb;
+              cp_async16(buf + stage_off<D>(rr, c), src, live);
             }
           };
 #pragma unroll
@@ -467,13 +485,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
             __syncwarp();
             if (sl < nh) {
               const float ws = exp2f(part_lse[pbase + sl] - M) * iw;
-              const uint32_t row = stage + (uint32_t)(sl % kMergeStages) * kMergeSlotBytes + lane * 256;
+              const uint32_t row = stage + (uint32_t)(sl % kMergeStages) * G::kMergeSlot;
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
+              for (int c = 0; c < G::kChunks; ++c) {
                 uint32_t w4[4];
                 asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
                              : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
-                             : "r"(row + ((c ^ (lane & 15)) << 4)));
+                             : "r"(row + stage_off<D>(lane, c)));
 #pragma unroll
                 for (int h2 = 0; h2 < 4; ++h2) {
                   const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[h2]));
@@ -487,12 +505,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           // out rows through the warp's (now idle) staging slot 0: two whole
           // rows per store instruction
 #pragma unroll
-          for (int e8 = 0; e8 < 16; ++e8)
-            st_shared_v4(stage + stage_off(lane, e8), pack_bf16x2(acc[8 * e8 + 0], acc[8 * e8 + 1]),
+          for (int e8 = 0; e8 < G::kChunks; ++e8)
+            st_shared_v4(stage + stage_off<D>(lane, e8), pack_bf16x2(acc[8 * e8 + 0], acc[8 * e8 + 1]),
                          pack_bf16x2(acc[8 * e8 + 2], acc[8 * e8 + 3]), pack_bf16x2(acc[8 * e8 + 4], acc[8 * e8 + 5]),
                          pack_bf16x2(acc[8 * e8 + 6], acc[8 * e8 + 7]));
           __syncwarp();
-          store_rows_from_stage(stage, out, (int64_t)r, valid, lane);
+          store_rows_from_stage<D>(stage, out, (int64_t)r, valid, lane);
           if (valid && lse != nullptr)
             lse[((size_t)b * dm.hq + h) * dm.N + t] = (M + log2f(W)) * kLn2;
         }
@@ -504,20 +522,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       const int y0 = b * dm.N + wk.key0;
-      const int x0 = g * kD;
+      const int x0 = g * D;
       int issued_k = 0, issued_v = 0;
       for (int i = 0; i < nkt; ++i) {
         const int s = i & 1;
-        const uint32_t ks = base + kOffK + s * kTile, vs = base + kOffV + s * kTile;
+        const uint32_t ks = base + G::kOffK + s * G::kTile, vs = base + G::kOffV + s * G::kTile;
         if (i >= 2 && !mbar_wait(bar(&ctl.k_free[s]), ((i >> 1) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(&ctl.k_full[s]), kTile);
-        tma_load_2d(ks, &tmK, x0, y0 + i * kBK, bar(&ctl.k_full[s]));
-        tma_load_2d(ks + kHalf, &tmK, x0 + 64, y0 + i * kBK, bar(&ctl.k_full[s]));
+        mbar_arrive_expect_tx(bar(&ctl.k_full[s]), G::kTile);
+#pragma unroll
+        for (int hh = 0; hh < G::kHalves; ++hh)
+          tma_load_2d(ks + hh * kHalf, &tmK, x0 + 64 * hh, y0 + i * kBK, bar(&ctl.k_full[s]));
         issued_k = i + 1;
         if (i >= 2 && !mbar_wait(bar(&ctl.v_free[s]), ((i >> 1) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(&ctl.v_full[s]), kTile);
-        tma_load_2d(vs, &tmV, x0, y0 + i * kBK, bar(&ctl.v_full[s]));
-        tma_load_2d(vs + kHalf, &tmV, x0 + 64, y0 + i * kBK, bar(&ctl.v_full[s]));
+        mbar_arrive_expect_tx(bar(&ctl.v_full[s]), G::kTile);
+#pragma unroll
+        for (int hh = 0; hh < G::kHalves; ++hh)
+          tma_load_2d(vs + hh * kHalf, &tmV, x0 + 64 * hh, y0 + i * kBK, bar(&ctl.v_full[s]));
         issued_v = i + 1;
       }
       if (*abort_flag) {
@@ -533,22 +553,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idS = idesc_bf16(128, kBK, false);
-      const uint32_t idO = idesc_bf16(128, kD, true);
+      const uint32_t idO = idesc_bf16(128, D, true);
       // descriptor words precomputed once; each MMA adds a compile-time offset
       const uint32_t hi = sdesc_hi(1024);
-      const uint32_t loQ = sdesc_lo(base + kOffQ, 16), loK = sdesc_lo(base + kOffK, 16),
-                     loV = sdesc_lo(base + kOffV, kHalf);
+      const uint32_t loQ = sdesc_lo(base + G::kOffQ, 16), loK = sdesc_lo(base + G::kOffK, 16),
+                     loV = sdesc_lo(base + G::kOffV, kHalf);
       auto issue_s = [&](int w, int s) {
-        const uint32_t qa = loQ + (w ? (kTile >> 4) : 0u), ka = loK + (s ? (kTile >> 4) : 0u);
+        const uint32_t qa = loQ + (w ? (G::kTile >> 4) : 0u), ka = loK + (s ? (G::kTile >> 4) : 0u);
         const uint32_t d = tb + (w ? 128u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
           mma_ss(d, sdesc_join(qa + off, hi), sdesc_join(ka + off, hi), idS, kk > 0);
         }
       };
       auto issue_pv = [&](int w, int s, bool acc) {
-        const uint32_t va = loV + (s ? (kTile >> 4) : 0u);
+        const uint32_t va = loV + (s ? (G::kTile >> 4) : 0u);
         const uint32_t d = tb + (w ? 384u : 256u), a = tb + (w ? 128u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -632,8 +652,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 bool make_kv_map(CUtensorMap* map, const void* base, const Dims& dm) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)dm.hkv * kD, (cuuint64_t)dm.batch * dm.N};
-  cuuint64_t strides[1] = {(cuuint64_t)dm.hkv * kD * 2};
+  cuuint64_t dims[2] = {(cuuint64_t)dm.hkv * dm.d, (cuuint64_t)dm.batch * dm.N};
+  cuuint64_t strides[1] = {(cuuint64_t)dm.hkv * dm.d * 2};
   cuuint32_t box[2] = {64, kBK};
   cuuint32_t es[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
@@ -644,16 +664,34 @@ bool make_kv_map(CUtensorMap* map, const void* base, const Dims& dm) {
 namespace {
 
 // the setmaxnreg split is only safe if the kernel really launches with kLaunchRegs
-template <int MODE>
+template <int MODE, int D>
 cudaError_t check_regs() {
   static int regs = -1;
   if (regs < 0) {
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, attn_tc_kernel<MODE>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_tc_kernel<MODE, D>);
     if (e != cudaSuccess) return e;
     regs = fa.numRegs;
   }
   return regs >= kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+template <int MODE, int D>
+cudaError_t launch_tc_d(const Dims& dm, const void* q, const void* k, const void* v,
+                        const int32_t* sel, const int32_t* offsets, const int32_t* rows,
+                        const AttnWs& ws, void* out, float* lse, int ch, int64_t grid,
+                        cudaStream_t stream) {
+  CUtensorMap mk, mv;
+  if (!make_kv_map(&mk, k, dm) || !make_kv_map(&mv, v, dm)) return cudaErrorInvalidValue;
+  cudaError_t e = check_regs<MODE, D>();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_tc_kernel<MODE, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Geo<D>::kSmem);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<MODE, D><<<grid, kThreads, Geo<D>::kSmem, stream>>>(
+      (const __nv_bfloat16*)q, mk, mv, sel, offsets, rows, ws.tile_start, ws.part_o, ws.part_lse,
+      (__nv_bfloat16*)out, lse, ws.status, dm, ch);
+  return cudaGetLastError();
 }
 
 template <int MODE>
@@ -661,22 +699,20 @@ cudaError_t launch_tc(const Dims& dm, const void* q, const void* k, const void* 
                       const int32_t* sel, const int32_t* offsets, const int32_t* rows,
                       const AttnWs& ws, void* out, float* lse, int ch, int64_t grid,
                       cudaStream_t stream) {
-  CUtensorMap mk, mv;
-  if (!make_kv_map(&mk, k, dm) || !make_kv_map(&mv, v, dm)) return cudaErrorInvalidValue;
-  cudaError_t e = check_regs<MODE>();
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmemBytes);
-  if (e != cudaSuccess) return e;
-  attn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, stream>>>(
-      (const __nv_bfloat16*)q, mk, mv, sel, offsets, rows, ws.tile_start, ws.part_o, ws.part_lse,
-      (__nv_bfloat16*)out, lse, ws.status, dm, ch);
-  return cudaGetLastError();
+  if (dm.d == 128)
+    return launch_tc_d<MODE, 128>(dm, q, k, v, sel, offsets, rows, ws, out, lse, ch, grid, stream);
+  if (dm.d == 64)
+    return launch_tc_d<MODE, 64>(dm, q, k, v, sel, offsets, rows, ws, out, lse, ch, grid, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 int attn_tc_rows_per_tile() { return kRowsPerCta; }
+
+// bf16 with head_dim 128 or 64 runs both attention steps on tcgen05 (with bf16
+// partial results); fp32 on the CUDA-core kernels
+bool attn_tc_path(int dtype, int d) { return dtype == MOBA_BF16 && (d == 128 || d == 64); }
 
 // the CTA-pair historical kernel (csrc/attn_pair_tc.cu) takes the same 256-row tiles
 bool attn_hist_pair_enabled();
@@ -687,7 +723,7 @@ cudaError_t launch_attn_pair_hist(const Dims& dm, const void* q, const void* k, 
 cudaError_t launch_attn_tc_hist(const Dims& dm, const void* q, const void* k, const void* v,
                                 const int32_t* sel, const int32_t* offsets, const int32_t* rows,
                                 const AttnWs& ws, int ch, int64_t grid, cudaStream_t stream) {
-  if (attn_hist_pair_enabled())
+  if (dm.d == 128 && attn_hist_pair_enabled())
     return launch_attn_pair_hist(dm, q, k, v, sel, offsets, rows, ws, ch, grid, stream);
   return launch_tc<kHist>(dm, q, k, v, sel, offsets, rows, ws, nullptr, nullptr, ch, grid, stream);
 }

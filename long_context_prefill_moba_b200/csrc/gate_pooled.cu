@@ -467,7 +467,7 @@ cudaError_t launch_attn_pooled(const Dims& dm, int dtype, const void* q, const v
   if (e != cudaSuccess) return e;
   const int KH = dm.topk - 1;
   // the partial outputs are bf16 for the tensor-core kernels, fp32 otherwise
-  const int part_elem_bytes = (dtype == MOBA_BF16 && dm.d == 128) ? 2 : 4;
+  const int part_elem_bytes = attn_tc_path(dtype, dm.d) ? 2 : 4;
   for (int ch = 0; ch < dm.nchunks; ++ch) {
     if (KH > 0) {
       const int t0 = ch * dm.chunk;

@@ -102,6 +102,9 @@ struct BwdWs {
   int32_t* tile_start;  // [b * hkv * n + 1] row-tile prefix of one pass (tensor-core path)
 };
 bool attn_bwd_tc_path(const Dims& dm, int dtype);
+// the forward attention steps run on tcgen05, with bf16 partial results
+// (bf16 with head_dim 128 or 64)
+bool attn_tc_path(int dtype, int d);
 cudaError_t launch_attn_bwd(const Dims& dm, int dtype, const void* q, const void* k, const void* v,
                             const void* out, const void* dout, const float* lse, const int32_t* sel,
                             const int32_t* offsets, const int32_t* rows, void* dq, void* dk, void* dv,

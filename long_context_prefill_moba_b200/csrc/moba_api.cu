@@ -25,9 +25,9 @@ int64_t chunk_of(const moba_shape_t* s) {
   const int64_t KH = s->topk - 1;
   if (KH == 0) return cap;
   // bytes of one partial result: bf16 output and fp32 log-sum-exp on the
-  // tensor-core path (bf16, head_dim 128), fp32 output and lse otherwise
-  const int64_t slot = s->dtype == MOBA_BF16 && s->head_dim == 128 ? 2 * s->head_dim + 4
-                                                                   : 4 * (s->head_dim + 1);
+  // tensor-core path (bf16, head_dim 128 or 64), fp32 output and lse otherwise
+  const int64_t slot = moba::attn_tc_path(s->dtype, s->head_dim) ? 2 * s->head_dim + 4
+                                                                 : 4 * (s->head_dim + 1);
   const int64_t per_token = (int64_t)s->batch * s->hq * KH * slot;
   int64_t c = 128;
   while (c * 2 <= cap && c * 2 * per_token <= kPartialBudget) c *= 2;
@@ -75,9 +75,9 @@ struct AttnLayout {
 AttnLayout attn_layout(const moba_shape_t* s) {
   const size_t KH = s->topk - 1;
   const size_t entries = (size_t)s->batch * chunk_of(s) * s->hq * KH;
-  // the tensor-core kernels (bf16, head_dim 128) keep the partial outputs in
-  // bf16; the others in fp32
-  const size_t part_bytes = s->dtype == MOBA_BF16 && s->head_dim == 128 ? 2 : 4;
+  // the tensor-core kernels (bf16, head_dim 128 or 64) keep the partial
+  // outputs in bf16; the others in fp32
+  const size_t part_bytes = moba::attn_tc_path(s->dtype, s->head_dim) ? 2 : 4;
   AttnLayout L;
   L.status = 0;
   L.part_o = 256;

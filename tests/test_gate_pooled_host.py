@@ -23,6 +23,7 @@ PROGRAM = r"""
 // the launchers gate_pooled.cu calls but this host program never runs
 namespace moba {
 bool gate_tc_pooled_supported(const Dims&, int) { return false; }
+bool attn_tc_path(int, int) { return false; }
 cudaError_t launch_gate_select_tc_pooled(const Dims&, int, int, const void*, const float*, const float*,
                                          const float*, int32_t*, int32_t*, int*, cudaStream_t) {
   return cudaErrorNotSupported;
