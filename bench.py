@@ -632,7 +632,10 @@ def main():
             "kernels_ms": {"meanpool": pool_ms, "gate": gate_ms, "attn": attn_ms},
             "roofline": {"bound": "tensor", "kernel": "moba_attn_fwd (attention + merge)",
                          "achieved": attn_tf, "peak": peak, "unit": "TFLOP/s", "frac": attn_tf / peak,
-                         "peak_kind": f"{peak_kind} bf16 sustained", "traffic": traffic,
+                         "peak_kind": f"{peak_kind} bf16 sustained", "peak_burst": peaks["bf16_tflops"],
+                         "frac_of_burst": attn_tf / peaks["bf16_tflops"],
+                         "peak_sustained_sm_mhz": peaks.get("clocks_under_load", {}).get("sm_mhz_median"),
+                         "traffic": traffic,
                          "traffic_note": traffic_note},
             "hbm_kernels": {
                 "meanpool": {"achieved": pool_bytes / (pool_ms * 1e-3) / 1e9, "unit": "GB/s",
