@@ -110,7 +110,9 @@ MOBA_DEV bool selectors_all(bool v, int wg) {
 }
 
 // ---- sorting networks on registers (descending) --------------------------------
-MOBA_DEV void cex(float& a, float& b) {
+// compiled for the host as well, so that a host program can check them
+#define MOBA_NET __host__ __device__ __forceinline__
+MOBA_NET void cex(float& a, float& b) {
   const float hi = fmaxf(a, b);
   b = fminf(a, b);
   a = hi;
@@ -151,17 +153,17 @@ static_assert(oem_pairs(16).n == 63 && oem_pairs(8).n == 19 && oem_pairs(4).n ==
 static_assert(bitonic_pairs(16).n == 32, "merger size");
 
 template <int K, bool Bitonic, size_t... I>
-MOBA_DEV void apply_pairs(float (&v)[K], std::index_sequence<I...>) {
+MOBA_NET void apply_pairs(float (&v)[K], std::index_sequence<I...>) {
   constexpr CePairs P = Bitonic ? bitonic_pairs(K) : oem_pairs(K);
   (cex(v[P.a[I]], v[P.b[I]]), ...);
 }
 template <int K>
-MOBA_DEV void sort_desc(float (&v)[K]) {
+MOBA_NET void sort_desc(float (&v)[K]) {
   apply_pairs<K, false>(v, std::make_index_sequence<oem_pairs(K).n>{});
 }
 // a <- the top K of a and b (both sorted descending), sorted descending
 template <int K>
-MOBA_DEV void merge_top(float (&a)[K], const float (&b)[K]) {
+MOBA_NET void merge_top(float (&a)[K], const float (&b)[K]) {
 #pragma unroll
   for (int i = 0; i < K; ++i) a[i] = fmaxf(a[i], b[K - 1 - i]);
   apply_pairs<K, true>(a, std::make_index_sequence<bitonic_pairs(K).n>{});
