@@ -74,7 +74,8 @@ typedef enum {
   MOBA_ERR_WORKSPACE = 3,    /* workspace smaller than the *_workspace_size  */
   MOBA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed         */
   MOBA_ERR_INTERNAL = 5,
-  MOBA_ERR_TIMEOUT = 6       /* reserved: a bounded device-side wait expired */
+  MOBA_ERR_TIMEOUT = 6       /* a bounded device-side wait expired; written to a
+                                device status word, never returned by a call    */
 } moba_status_t;
 
 typedef enum { MOBA_BF16 = 0, MOBA_F32 = 1 } moba_dtype_t;
