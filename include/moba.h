@@ -44,8 +44,9 @@
  *   - seqlen need not be a multiple of block: the last block is shorter.
  *   - scale <= 0 selects 1/sqrt(head_dim).  lse is the natural-log
  *     log-sum-exp of the scaled logits.
- *   - Sizes: seqlen*hq*batch < 2^31 and head_dim in {64, 128};
- *     1 <= topk <= MOBA_MAX_TOPK.
+ *   - Sizes: seqlen*hq*batch < 2^31, head_dim in {64, 128},
+ *     1 <= topk <= MOBA_MAX_TOPK, and at most 65535 blocks and 65535 batch
+ *     entries (MOBA_ERR_UNSUPPORTED beyond).
  */
 #ifndef MOBA_H_
 #define MOBA_H_

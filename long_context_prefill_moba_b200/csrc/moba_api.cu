@@ -10,6 +10,7 @@ thread_local int g_last_cuda_error = 0;
 thread_local int g_last_launches = 0;
 
 constexpr int64_t kI32Max = 2147483647;
+constexpr int64_t kGridYZMax = 65535;            // largest y or z extent of a CUDA grid
 constexpr int64_t kPartialBudget = 8ll << 30;   // bytes of partials per pass (automatic chunk)
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -139,6 +140,8 @@ MOBA_API moba_status_t moba_check_shape(const moba_shape_t* s) {
     return MOBA_ERR_INVALID_ARG;
   if (s->head_dim != 64 && s->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
   if (s->topk > MOBA_MAX_TOPK) return MOBA_ERR_UNSUPPORTED;
+  // the pooling kernels put blocks and batch entries on the grid's y and z axes
+  if (nblocks(s) > kGridYZMax || s->batch > kGridYZMax) return MOBA_ERR_UNSUPPORTED;
   if ((int64_t)s->batch * s->seqlen * s->hq > kI32Max) return MOBA_ERR_UNSUPPORTED;
   if (rows_total(s) > kI32Max) return MOBA_ERR_UNSUPPORTED;
   if (ngroups_total(s) + 1 > kI32Max) return MOBA_ERR_UNSUPPORTED;

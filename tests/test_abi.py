@@ -70,6 +70,12 @@ def test_sizes_of_the_1m_layer(L):
     assert M.moba_gate_workspace_size(s) >= 2 * 4 * M.moba_num_chunks(s) * 8 * 256
 
 
+def test_largest_block_count_accepted(L):
+    s = shape(seqlen=65535 * 16, hq=1, hkv=1, block=16, topk=2)
+    assert M.moba_check_shape(s) == 0 and M.moba_num_blocks(s) == 65535
+    assert M.moba_check_shape(shape(seqlen=65535 * 16 + 1, hq=1, hkv=1, block=16, topk=2)) == 2
+
+
 def test_rows_count_ragged_and_small(L):
     s = shape(batch=2, seqlen=1000, hq=4, hkv=2, block=96, topk=3)
     exact = sum(min(2, t // 96) for t in range(1000)) * 2 * 4
@@ -83,6 +89,7 @@ def test_rows_count_ragged_and_small(L):
     (dict(topk=0), 1), (dict(dtype="f32", head_dim=96), 2), (dict(topk=17), 2),
     (dict(query_chunk=100), 1), (dict(scale=float("nan")), 1),
     (dict(batch=64, seqlen=1 << 20, hq=64), 2),
+    (dict(seqlen=1 << 20, hq=1, hkv=1, block=8), 2),      # 131072 blocks: more than a grid axis holds
 ])
 def test_invalid_shapes_rejected(L, kw, status):
     s = shape(**kw)
