@@ -322,8 +322,9 @@ def config_of(cfg, args):
 
 
 # ---------------------------------------------------------------------------
-# Speed-up curve: MoBA layer vs dense causal attention at growing lengths
-# (the comparison of the paper's Figure 2a, on this GPU)
+# Other modes: the backward, the pooled-gate variant, and the speed-up curve
+# (MoBA layer vs dense causal attention at growing lengths: the comparison of
+# the paper's Figure 2a, on this GPU)
 # ---------------------------------------------------------------------------
 def backward_bench(cfg, steps, warmup):
     """One JSON line: the attention backward (moba_attn_bwd: dq, dk, dv given a
